@@ -1,0 +1,7 @@
+"""Oracle package (TEST INFRASTRUCTURE): plain fp64 CPU statement of the method.
+
+Only tests/, __graft_entry__.smoke() and bench.py's CPU-baseline and
+reference legs may import it.  See ``oracle.expert`` for the cited passages.
+"""
+
+from . import expert  # noqa: F401

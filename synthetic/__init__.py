@@ -1,0 +1,21 @@
+"""Seeded synthetic inputs shared by the oracle and the CUDA path.
+
+This module only draws random numbers and lays them out: workload shapes,
+per-tensor seeded normal draws, and the bf16 storage rounding of inputs that
+are *given* in bf16.  It holds none of the method's arithmetic (no norm, no
+attention, no time embedding, no Euler step), so the oracle and the CUDA
+path can both use it without sharing any computation.
+"""
+
+from .configs import CONFIGS, ExpertShape, get_config  # noqa: F401
+from .gen import (  # noqa: F401
+    bf16_bits_to_f32,
+    f32_to_bf16_bits,
+    make_draft,
+    make_noise,
+    make_prefix_kv,
+    make_state,
+    make_weights,
+    round_to_bf16,
+    weight_names,
+)

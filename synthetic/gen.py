@@ -1,0 +1,151 @@
+"""Seeded tensor generation.
+
+Every tensor has its own stream: ``numpy.random.PCG64`` seeded with
+``SeedSequence([seed, crc32(tensor name)])``, drawn with ``standard_normal``
+in float32 and scaled by the tensor's standard deviation.  Adding or
+removing a tensor therefore never changes another tensor's values.
+
+Distributions (the workloads' stand-ins for the pages' real checkpoints and
+camera/robot data, which are not available):
+  * every weight matrix, bias and norm gain ~ N(0, 0.02)
+  * prefix KV cache ~ N(0, 1)
+  * noise eps ~ N(0, 1), robot state ~ N(0, 1)
+  * FLASH draft chunk ~ N(0, 0.5) with the gripper dim set to +-1 and 0 or 1
+    sign switch at a seeded row
+
+bf16 inputs are produced by round-to-nearest-even of the float32 draw; both
+the oracle and the CUDA path receive the same rounded values.
+"""
+
+from __future__ import annotations
+
+import zlib
+from typing import Dict, List, Tuple
+
+import numpy as np
+
+from .configs import ExpertShape
+
+
+def _rng(seed: int, name: str) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, zlib.crc32(name.encode())])))
+
+
+def _normal(seed: int, name: str, shape, std: float) -> np.ndarray:
+    a = _rng(seed, name).standard_normal(size=shape, dtype=np.float32)
+    if std != 1.0:
+        a *= np.float32(std)
+    return a
+
+
+# ---------------------------------------------------------------------------
+# bf16 storage format (IEEE binary32 with the low 16 bits dropped after
+# round-to-nearest-even).  Used only to produce inputs that are given in bf16.
+# ---------------------------------------------------------------------------
+
+def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """Round float32 values to bf16 (nearest-even); return the uint16 bit patterns."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    lsb = (u >> np.uint32(16)) & np.uint32(1)
+    r = (u + np.uint32(0x7FFF) + lsb) >> np.uint32(16)
+    return r.astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def round_to_bf16(a: np.ndarray) -> np.ndarray:
+    """float32 array holding the bf16-rounded values of ``a``."""
+    return bf16_bits_to_f32(f32_to_bf16_bits(a))
+
+
+# ---------------------------------------------------------------------------
+# weights
+# ---------------------------------------------------------------------------
+
+def weight_names(cfg: ExpertShape) -> List[Tuple[str, Tuple[int, ...]]]:
+    """(name, shape) of every expert parameter, matrices as [out][in]."""
+    w, a, sd, f = cfg.width, cfg.action_dim, cfg.state_dim, cfg.mlp_dim
+    out = [
+        ("state_proj.w", (w, sd)), ("state_proj.b", (w,)),
+        ("action_in_proj.w", (w, a)), ("action_in_proj.b", (w,)),
+        ("time_mlp_in.w", (w, w)), ("time_mlp_in.b", (w,)),
+        ("time_mlp_out.w", (w, w)), ("time_mlp_out.b", (w,)),
+    ]
+    for l in range(cfg.n_layers):
+        p = f"layers.{l}."
+        out += [
+            (p + "attn_norm.g", (w,)),
+            (p + "q_proj.w", (cfg.q_dim, w)),
+            (p + "k_proj.w", (cfg.kv_dim, w)),
+            (p + "v_proj.w", (cfg.kv_dim, w)),
+            (p + "o_proj.w", (w, cfg.q_dim)),
+            (p + "mlp_norm.g", (w,)),
+            (p + "gate_proj.w", (f, w)),
+            (p + "up_proj.w", (f, w)),
+            (p + "down_proj.w", (w, f)),
+        ]
+    out += [("final_norm.g", (w,)), ("action_out_proj.w", (a, w)), ("action_out_proj.b", (a,))]
+    return out
+
+
+def make_weights(cfg: ExpertShape, seed: int | None = None) -> Dict[str, np.ndarray]:
+    """All expert parameters as float32 arrays.
+
+    In a "bf16" workload every 2-D matrix holds bf16-representable values
+    (it is stored and streamed as bf16); 1-D biases and gains stay float32.
+    """
+    seed = cfg.seed if seed is None else seed
+    ws: Dict[str, np.ndarray] = {}
+    for name, shape in weight_names(cfg):
+        a = _normal(seed, name, shape, cfg.weight_std)
+        if cfg.dtype == "bf16" and len(shape) == 2:
+            a = round_to_bf16(a)
+        ws[name] = a
+    return ws
+
+
+def make_prefix_kv(cfg: ExpertShape, batch: int | None = None, prefix_len: int | None = None,
+                   seed: int | None = None) -> np.ndarray:
+    """Prefix KV cache [L][2][B][P][Hkv][D] ~ N(0,1) (bf16 values in a bf16 workload)."""
+    seed = cfg.seed if seed is None else seed
+    b = cfg.batch if batch is None else batch
+    p = cfg.prefix_len if prefix_len is None else prefix_len
+    kv = _normal(seed, "prefix_kv", (cfg.n_layers, 2, b, p, cfg.n_kv_heads, cfg.head_dim), 1.0)
+    if cfg.dtype == "bf16":
+        kv = round_to_bf16(kv)
+    return kv
+
+
+def make_noise(cfg: ExpertShape, batch: int | None = None, seed: int | None = None,
+               name: str = "noise") -> np.ndarray:
+    """eps ~ N(0,1), [B][H][A] float32."""
+    seed = cfg.seed if seed is None else seed
+    b = cfg.batch if batch is None else batch
+    return _normal(seed, name, (b, cfg.chunk_len, cfg.action_dim), 1.0)
+
+
+def make_state(cfg: ExpertShape, batch: int | None = None, seed: int | None = None) -> np.ndarray:
+    """Robot state ~ N(0,1), [B][Sd] float32."""
+    seed = cfg.seed if seed is None else seed
+    b = cfg.batch if batch is None else batch
+    return _normal(seed, "state", (b, cfg.state_dim), 1.0)
+
+
+def make_draft(cfg: ExpertShape, n_switch: int = 0, seed: int | None = None) -> np.ndarray:
+    """FLASH candidate chunk D [H][A] ~ N(0, draft_std); gripper dim in {-1,+1}.
+
+    ``n_switch`` = 0: the gripper keeps one seeded sign over the chunk.
+    ``n_switch`` = 1: the sign flips once, at a seeded row r in [1, H).
+    """
+    seed = cfg.seed if seed is None else seed
+    d = _normal(seed, "draft", (cfg.chunk_len, cfg.action_dim), cfg.draft_std)
+    rng = _rng(seed, "draft_gripper")
+    sign0 = np.float32(1.0 if rng.integers(0, 2) else -1.0)
+    g = np.full(cfg.chunk_len, sign0, dtype=np.float32)
+    if n_switch:
+        r = int(rng.integers(1, cfg.chunk_len))
+        g[r:] = -sign0
+    d[:, cfg.gripper] = g
+    return d

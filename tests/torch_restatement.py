@@ -1,0 +1,93 @@
+"""An independent second statement of the action expert in PyTorch (CPU, float64).
+
+Used only to cross-check the oracle.  It is written in a different style on
+purpose -- all suffixes batched, torch.nn.functional's rms_norm / gelu /
+silu / scaled_dot_product_attention with an explicit boolean mask, a
+complex-number RoPE -- so that a slip in one statement (a transposed
+operand, a dropped term, a wrong pairing) shows up as a disagreement.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+
+T64 = torch.float64
+
+
+def _t(a):
+    return torch.as_tensor(np.asarray(a), dtype=T64)
+
+
+def time_cond(W, t, width):
+    half = width // 2
+    expo = torch.linspace(0.0, 1.0, half, dtype=T64)
+    period = 4e-3 * torch.pow(torch.tensor(4.0 / 4e-3, dtype=T64), expo)
+    ang = 2 * math.pi * t / period
+    e = torch.cat([torch.sin(ang), torch.cos(ang)])
+    z = F.linear(e, _t(W["time_mlp_in.w"]), _t(W["time_mlp_in.b"]))
+    return F.linear(F.silu(z), _t(W["time_mlp_out.w"]), _t(W["time_mlp_out.b"]))
+
+
+def rope_complex(x, pos, theta):
+    """x [..., S, heads, D]; rotate pairs (d, d+D/2) as complex numbers d + i(d+D/2)."""
+    if theta == 0:
+        return x
+    d = x.shape[-1]
+    half = d // 2
+    freqs = 1.0 / (theta ** (torch.arange(0, half, dtype=T64) * 2.0 / d))
+    ang = pos.to(T64)[:, None] * freqs[None, :]            # [S, half]
+    rot = torch.polar(torch.ones_like(ang), ang)[:, None, :]  # [S, 1, half]
+    z = torch.complex(x[..., :half], x[..., half:]) * rot
+    return torch.cat([z.real, z.imag], dim=-1)
+
+
+def velocity(W, cfg, x_t, state, t, prefix_k, prefix_v):
+    """v [G][H][A] for G suffixes sharing one prefix; t is a per-suffix sequence.
+
+    x_t [G][H][A], state [Sd], prefix_k/v [L][P][Hkv][D]."""
+    x_t = _t(x_t)
+    g_count, h_len, _ = x_t.shape
+    s_len = h_len + 1
+    p_len = prefix_k.shape[1]
+    hq, hkv, d = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim
+    w = cfg.width
+    eps = cfg.rms_eps
+
+    st = F.linear(_t(state), _t(W["state_proj.w"]), _t(W["state_proj.b"]))
+    act = F.linear(x_t, _t(W["action_in_proj.w"]), _t(W["action_in_proj.b"]))
+    c = torch.stack([time_cond(W, float(tt), w) for tt in t])      # [G, w]
+    h = torch.cat([st.expand(g_count, 1, w), act + c[:, None, :]], dim=1)  # [G, S, w]
+
+    pos = torch.arange(p_len, p_len + s_len)
+    mask = torch.ones(s_len, p_len + s_len, dtype=torch.bool)
+    if cfg.suffix_mask == "pi0_block":
+        mask[0, p_len + 1:] = False
+
+    for l in range(cfg.n_layers):
+        p = f"layers.{l}."
+        u = F.rms_norm(h, (w,), weight=1.0 + _t(W[p + "attn_norm.g"]), eps=eps)
+        q = F.linear(u, _t(W[p + "q_proj.w"])).view(g_count, s_len, hq, d)
+        k = F.linear(u, _t(W[p + "k_proj.w"])).view(g_count, s_len, hkv, d)
+        v = F.linear(u, _t(W[p + "v_proj.w"])).view(g_count, s_len, hkv, d)
+        q = rope_complex(q, pos, cfg.rope_theta)
+        k = rope_complex(k, pos, cfg.rope_theta)
+        pk = _t(prefix_k[l]).expand(g_count, p_len, hkv, d)
+        pv = _t(prefix_v[l]).expand(g_count, p_len, hkv, d)
+        keys = torch.cat([pk, k], dim=1).transpose(1, 2)     # [G, Hkv, keys, D]
+        vals = torch.cat([pv, v], dim=1).transpose(1, 2)
+        rep = hq // hkv
+        keys = keys.repeat_interleave(rep, dim=1)
+        vals = vals.repeat_interleave(rep, dim=1)
+        o = F.scaled_dot_product_attention(q.transpose(1, 2), keys, vals, attn_mask=mask)
+        o = o.transpose(1, 2).reshape(g_count, s_len, hq * d)
+        h = h + F.linear(o, _t(W[p + "o_proj.w"]))
+        u = F.rms_norm(h, (w,), weight=1.0 + _t(W[p + "mlp_norm.g"]), eps=eps)
+        gate = F.gelu(F.linear(u, _t(W[p + "gate_proj.w"])), approximate="tanh")
+        h = h + F.linear(gate * F.linear(u, _t(W[p + "up_proj.w"])), _t(W[p + "down_proj.w"]))
+
+    hf = F.rms_norm(h[:, 1:], (w,), weight=1.0 + _t(W["final_norm.g"]), eps=eps)
+    return F.linear(hf, _t(W["action_out_proj.w"]), _t(W["action_out_proj.b"])).numpy()
