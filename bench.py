@@ -1,0 +1,359 @@
+#!/usr/bin/env python
+"""Benchmark: latency of one 10-step action chunk of the pi0-class bf16 action
+expert (18 layers, width 1024, 8 q / 1 kv heads, head_dim 256, GeGLU 4096,
+816-token prefix KV, 1 state + 50 action tokens, batch 1), and the HBM
+bandwidth it achieves.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One "step" is one call of rtv_denoise: the whole hot path (10 Euler steps
+through the expert) over one batch of synthetic input.  With N > 1 the
+script is launched by torchrun, one process per GPU; every rank runs an
+independent replica (weak scaling, no data-path collective) and the time is
+the max over ranks.  Rank 0 prints one JSON line.
+
+Timing: W untimed warm-up calls, then K calls bracketed by a barrier and a
+device synchronise, timed with CUDA events on the launching stream.  The
+expert's 623 MB of weights stream from HBM on every step (L2 is 126 MB), so
+no separate L2 flush is done.  `e2e` repeats the measurement through the C
+ABI with pinned host buffers, the host<->device copies inside the timed
+region.  `cpu_baseline` times the CPU oracle on a bounded sample.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "10-step action-chunk latency (us) and achieved HBM GB/s vs 8 TB/s roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="pi0-bf16")
+    ap.add_argument("--n-steps", type=int, default=10, help="Euler steps per chunk")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds of the oracle sample")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes
+# ---------------------------------------------------------------------------
+
+def algorithmic_bytes_per_step(cfg, batch=1):
+    """Weight bytes of every layer and of the state/action projections, plus
+    the prefix K and V of every layer, each counted once per Euler step.
+    The time MLP depends only on t and is precomputed, so it is excluded."""
+    elt = 4 if cfg.dtype == "f32" else 2
+    w, f = cfg.width, cfg.mlp_dim
+    mlp_elt = 1 if cfg.mlp_dtype == "fp8_e4m3" else elt
+    attn = w * (cfg.q_dim + 2 * cfg.kv_dim) + cfg.q_dim * w
+    layer = attn * elt + 3 * w * f * mlp_elt
+    proj = (w * cfg.state_dim + w * cfg.action_dim + cfg.action_dim * w) * elt
+    kv = 2 * batch * cfg.prefix_len * cfg.kv_dim * elt
+    return cfg.n_layers * (layer + kv) + proj
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clock sampling during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline and reference arm)
+# ---------------------------------------------------------------------------
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_step_seconds(cfg, target_s: float, min_samples: int = 1, max_samples: int = 10):
+    """Seconds per Euler step of the CPU oracle on the workload (bounded sample)."""
+    from oracle import expert as O
+    from synthetic import make_noise, make_prefix_kv, make_state, make_weights
+    W = O.to_f64(make_weights(cfg))
+    kv = make_prefix_kv(cfg)
+    x = make_noise(cfg)[0].astype(np.float64)
+    state = make_state(cfg)[0]
+    pk, pv = kv[:, 0, 0].astype(np.float64), kv[:, 1, 0].astype(np.float64)
+    times = []
+    t_total = 0.0
+    k = 0
+    while (k < min_samples or t_total < target_s) and k < max_samples:
+        t = 1.0 - (k % cfg.n_steps) / cfg.n_steps
+        t0 = time.perf_counter()
+        v = O.expert_velocity(W, cfg, x, state, t, pk, pv)
+        x = x - v / cfg.n_steps
+        dt = time.perf_counter() - t0
+        times.append(dt)
+        t_total += dt
+        k += 1
+    return statistics.median(times), k
+
+
+def run_reference(args, info):
+    """The CPU oracle, as it stands, on a bounded sample of the workload:
+    each step is one Euler step of the chunk, scaled to chunk latency."""
+    if not info.is_main:
+        return
+    from synthetic import get_config
+    cfg = get_config(args.workload, n_steps=args.n_steps)
+    from oracle import expert as O
+    from synthetic import make_noise, make_prefix_kv, make_state, make_weights
+    W = O.to_f64(make_weights(cfg))
+    kv = make_prefix_kv(cfg)
+    pk, pv = kv[:, 0, 0].astype(np.float64), kv[:, 1, 0].astype(np.float64)
+    x = make_noise(cfg)[0].astype(np.float64)
+    state = make_state(cfg)[0]
+    for _ in range(max(0, min(args.warmup, 1))):
+        O.expert_velocity(W, cfg, x, state, 1.0, pk, pv)
+    steps = max(1, min(args.steps, 20))
+    t0 = time.perf_counter()
+    for k in range(steps):
+        t = 1.0 - (k % cfg.n_steps) / cfg.n_steps
+        x = x - O.expert_velocity(W, cfg, x, state, t, pk, pv) / cfg.n_steps
+    per_step = (time.perf_counter() - t0) / steps
+    chunk_us = per_step * cfg.n_steps * 1e6
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": chunk_us, "unit": "us", "n_gpus": args.gpus,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": chunk_us / 1000.0, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "n_steps": cfg.n_steps, "batch": 1, "prefix_len": cfg.prefix_len},
+        "cpu_baseline": {"value": chunk_us, "unit": "us", "cores": cores, "kind": "oracle",
+                         "sample": f"{steps} single Euler steps of the {args.workload} chunk (fp64 numpy oracle), "
+                                   f"each scaled x{cfg.n_steps} to chunk latency"},
+        "e2e": {"value": chunk_us, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, info):
+    import torch
+
+    from flow_matching_action_dm0_b200 import ActionExpert
+    from flow_matching_action_dm0_b200 import replicas as R
+    from synthetic import f32_to_bf16_bits, get_config, make_noise, make_prefix_kv, make_state, make_weights
+
+    dev = info.local_rank
+    torch.cuda.set_device(dev)
+    cfg = get_config(args.workload, n_steps=args.n_steps)
+    weights = make_weights(cfg)
+    kv = make_prefix_kv(cfg)
+    noise = make_noise(cfg)
+    state = make_state(cfg)
+
+    ex = ActionExpert(cfg, device=dev, max_batch=cfg.batch, max_taus=4)
+    ex.load(weights)
+    del weights
+    if cfg.dtype == "bf16":
+        kv_t = torch.from_numpy(f32_to_bf16_bits(kv).view(np.int16)).view(torch.bfloat16).cuda(dev)
+    else:
+        kv_t = torch.from_numpy(kv).cuda(dev)
+    stream = torch.cuda.Stream(dev)
+    ex.set_prefix_kv(kv_t, stream=stream)
+    noise_d = torch.from_numpy(noise).cuda(dev)
+    state_d = torch.from_numpy(state).cuda(dev)
+    out_d = torch.empty_like(noise_d)
+    torch.cuda.synchronize(dev)
+
+    n = cfg.n_steps
+    for _ in range(max(3, args.warmup)):
+        ex.denoise(noise_d, state_d, n, out_d, stream=stream)
+    torch.cuda.synchronize(dev)
+    s, bits = ex.status()
+    if s != 0:
+        raise RuntimeError(f"device status {bits:#x} after warm-up")
+
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    gpu_id = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    K = args.steps
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    R.barrier(info, dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(gpu_id) as clk:
+        start.record(stream)
+        for _ in range(K):
+            ex.denoise(noise_d, state_d, n, out_d, stream=stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    R.barrier(info, dev)
+    ms_local = start.elapsed_time(end) / K
+    ms = R.max_over_ranks(ms_local, info, dev)
+    s, bits = ex.status()
+    if s != 0:
+        raise RuntimeError(f"device status {bits:#x} after the timed region")
+
+    # end to end through the C ABI with pinned host buffers
+    noise_h = torch.from_numpy(noise).pin_memory()
+    state_h = torch.from_numpy(state).pin_memory()
+    out_h = torch.empty_like(noise_h).pin_memory()
+    for _ in range(2):
+        ex.denoise(noise_h, state_h, n, out_h, stream=stream)
+    torch.cuda.synchronize(dev)
+    R.barrier(info, dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        ex.denoise(noise_h, state_h, n, out_h, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    R.barrier(info, dev)
+    e2e_ms = R.max_over_ranks(e0.elapsed_time(e1) / K, info, dev)
+
+    launches_per_call = ex.kernels_per_call(n)
+    path = ex.path
+    ex.close()
+
+    if not info.is_main:
+        return
+    peaks, peak_kind = load_peaks()
+    bytes_step = algorithmic_bytes_per_step(cfg)
+    bytes_chunk = bytes_step * n
+    achieved = bytes_chunk / (ms * 1e-3) / 1e9
+    peak = float(peaks["hbm_gbs"])
+    line = {
+        "metric": METRIC,
+        "value": ms * 1000.0,
+        "unit": "us",
+        "n_gpus": info.world,
+        "steps": K,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": ms,
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": cfg.dtype,
+        "data": "synthetic",
+        "config": {"workload": args.workload, "n_steps": n, "batch": cfg.batch, "prefix_len": cfg.prefix_len,
+                   "layers": cfg.n_layers, "width": cfg.width, "parallelism": f"replicas x{info.world}",
+                   "l2": "inputs larger than L2: 623 MB of weights stream from HBM every Euler step; no flush",
+                   "path": path},
+        "chunks_per_s": info.world * 1000.0 / ms,
+        "roofline": {"bound": "hbm", "kernel": "whole denoise graph (all kernels of one chunk)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_kind": f"{peak_kind} hbm_gbs", "algorithmic_bytes_per_launch": bytes_chunk,
+                     "traffic": None},
+        "e2e": {"value": e2e_ms * 1000.0, "unit": "us",
+                "h2d_bytes_per_step": int(noise.nbytes + state.nbytes), "d2h_bytes_per_step": int(noise.nbytes)},
+        "clocks": clk.summary(),
+        "gpu_launches": int(launches_per_call * K) if launches_per_call > 0 else None,
+    }
+    if info.world == 1 and not args.no_cpu_baseline:
+        per_step_s, k = oracle_step_seconds(cfg, args.cpu_seconds)
+        line["cpu_baseline"] = {
+            "value": per_step_s * n * 1e6, "unit": "us", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{k} single Euler steps of the {args.workload} chunk (fp64 numpy oracle, median), "
+                      f"scaled x{n} to one chunk"}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    from flow_matching_action_dm0_b200 import replicas as R
+    info = R.rank_info()
+    if args.impl == "reference":
+        if info.world > 1 and not info.is_main:
+            return 0
+        run_reference(args, info)
+        return 0
+    info = R.init("nccl" if info.world > 1 else "gloo")
+    try:
+        run_ours(args, info)
+    finally:
+        R.shutdown(info)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

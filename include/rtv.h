@@ -1,0 +1,195 @@
+/*
+ * rtv.h -- C ABI of a B200 (sm_100a) implementation of the flow-matching
+ * action-expert suffix loop of a Pi0/DM0.5-class VLA, and of FLASH parallel
+ * verification.
+ *
+ * Pages (cited by title and section):
+ *   [DM0.5] "DM0.5: high-performance embodied VLA and OpenDM reading guide"
+ *           sec. 5.1 prefix encoded once into a per-layer KV cache,
+ *           sec. 5.2 action expert (action_in_proj, time_mlp_in/out, prefix
+ *           KV access, action_out_proj -> velocity), sec. 5.3 flow matching
+ *           and Euler sampling (diffusion_steps = 10, action chunk),
+ *           sec. 6.1 fixed image-count / static I/O contract, sec. 6.5
+ *           startup graph capture with static addresses, one replay, step
+ *           count fixed at capture.
+ *   [FLASH] "Realtime-VLA FLASH" sec. 02 (interpolate, predict, rebuild the
+ *           endpoint, compare), sec. 03.2 (accept the prefix below delta at
+ *           every verification time; zero length -> full path), sec. 03.3
+ *           (gripper switch -> full path).
+ *
+ * Conventions shared by every call:
+ *   - Matrices are row-major [out][in].  Activations and actions are fp32.
+ *   - Work is enqueued on the caller's stream and is asynchronous; outputs
+ *     are valid once that stream has completed.  Calls on one context must
+ *     not run concurrently from several host threads.
+ *   - Errors detectable on the host return at once and enqueue nothing.
+ *     Errors raised by kernels (a bounded wait that gave up, a non-finite
+ *     result) set bits of a device status word, read by rtv_device_status.
+ *   - No exception or abort crosses this boundary.  rtv_last_error gives a
+ *     one-line description of the last failure on the context.
+ *   - Pointers are owned by the caller unless stated.  The library copies
+ *     what it keeps (weights, prefix KV) into memory it owns.
+ */
+#ifndef RTV_H
+#define RTV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+/* A CUDA stream (cudaStream_t).  NULL means the legacy default stream. */
+typedef struct CUstream_st* rtv_stream;
+
+typedef enum {
+  RTV_OK = 0,
+  RTV_ERR_ARG = 1,         /* null pointer, bad enum, bad name or size        */
+  RTV_ERR_SHAPE = 2,       /* shape differs from the config or exceeds a max  */
+  RTV_ERR_STATE = 3,       /* call order: e.g. denoise before load/prefix     */
+  RTV_ERR_CUDA = 4,        /* a CUDA runtime call failed                      */
+  RTV_ERR_OOM = 5,         /* device allocation failed                        */
+  RTV_ERR_TIMEOUT = 6,     /* a device-side bounded wait gave up              */
+  RTV_ERR_NUMERIC = 7,     /* non-finite value detected on the device        */
+  RTV_ERR_UNSUPPORTED = 8  /* valid request this build does not implement     */
+} rtv_status;
+
+typedef enum { RTV_F32 = 0, RTV_BF16 = 1, RTV_FP8_E4M3 = 2, RTV_SAME = 3 } rtv_dtype;
+
+typedef enum {
+  RTV_MASK_BIDIR = 0,      /* every suffix token sees the prefix and its whole suffix */
+  RTV_MASK_PI0_BLOCK = 1   /* the state token does not see the action tokens          */
+} rtv_suffix_mask;
+
+/* Device status bits (rtv_device_status). */
+#define RTV_DEV_TIMEOUT  0x1u   /* a bounded spin-wait in a kernel gave up   */
+#define RTV_DEV_NUMERIC  0x2u   /* a NaN/Inf reached the action output       */
+#define RTV_DEV_BOUNDS   0x4u   /* a kernel's own index check refused work   */
+
+/* Verification flags ([FLASH] 03.2-03.3). */
+#define RTV_FLAG_ZERO_ACCEPT      0x1u  /* accepted length 0 -> full path               */
+#define RTV_FLAG_SWITCH           0x2u  /* gripper sign switch in the candidate chunk  */
+#define RTV_FLAG_SWITCH_IN_PREFIX 0x4u  /* a switch lies inside the accepted prefix    */
+
+/*
+ * Expert shape and settings.  [DM0.5] 5.2: a Gemma-style action expert of
+ * n_layers layers, hidden width `width`, grouped-query attention with
+ * n_q_heads query heads sharing n_kv_heads key/value heads of head_dim, a
+ * gated (GeGLU) MLP of mlp_dim; a suffix of one state token (state_dim) and
+ * chunk_len action tokens (action_dim) attends to a cached prefix of up to
+ * max_prefix_len tokens per layer.
+ *
+ * dtype (RTV_F32 or RTV_BF16) is the storage and tensor-core input type of
+ * the weight matrices and of the prefix KV; biases and norm gains are fp32.
+ * mlp_dtype: RTV_SAME, or RTV_FP8_E4M3 for gate/up/down weights stored in
+ * E4M3 with one fp32 scale per output row ([DM0.5] 6.3).
+ * rope_theta 0 disables rotary embedding.  barrier_timeout_ns bounds every
+ * device-side wait (0 = library default, 100 ms).
+ */
+typedef struct {
+  int n_layers, width, n_q_heads, n_kv_heads, head_dim, mlp_dim;
+  int action_dim, state_dim, chunk_len;
+  int max_prefix_len, max_batch, max_taus;
+  int dtype;
+  int mlp_dtype;
+  int suffix_mask;
+  float rms_eps;
+  float rope_theta;
+  long long barrier_timeout_ns;
+} rtv_expert_config;
+
+/*
+ * One named parameter for rtv_load_expert.  `data` points to host memory
+ * (is_device = 0) or device memory (is_device = 1) holding a dense
+ * row-major array of `shape` in `dtype`.  Names and shapes (w = width,
+ * A = action_dim, Sd = state_dim, F = mlp_dim, Q = n_q_heads*head_dim,
+ * KV = n_kv_heads*head_dim, l = layer index):
+ *   state_proj.w [w][Sd]  state_proj.b [w]
+ *   action_in_proj.w [w][A]  action_in_proj.b [w]
+ *   time_mlp_in.w [w][w]  time_mlp_in.b [w]  time_mlp_out.w [w][w]  time_mlp_out.b [w]
+ *   layers.l.attn_norm.g [w]  layers.l.q_proj.w [Q][w]  layers.l.k_proj.w [KV][w]
+ *   layers.l.v_proj.w [KV][w] layers.l.o_proj.w [w][Q]  layers.l.mlp_norm.g [w]
+ *   layers.l.gate_proj.w [F][w]  layers.l.up_proj.w [F][w]  layers.l.down_proj.w [w][F]
+ *   layers.l.gate_proj.s [F]  layers.l.up_proj.s [F]  layers.l.down_proj.s [w]
+ *        (fp32 per-row scales, only with mlp_dtype = RTV_FP8_E4M3)
+ *   final_norm.g [w]  action_out_proj.w [A][w]  action_out_proj.b [A]
+ * Matrices must be given in the config dtype (or RTV_FP8_E4M3 for the MLP
+ * when mlp_dtype says so); vectors in RTV_F32.
+ */
+typedef struct {
+  const char* name;
+  const void* data;
+  int dtype;
+  int ndim;
+  long long shape[4];
+  int is_device;
+} rtv_tensor;
+
+typedef struct rtv_ctx rtv_ctx;
+
+/* Create a context on CUDA device `cuda_device`; allocates the static
+ * buffers for the config's maxima.  *out is NULL on failure. */
+rtv_status rtv_create(const rtv_expert_config* cfg, int cuda_device, rtv_ctx** out);
+
+/* Copy and pack the expert's parameters ([DM0.5] 5.2).  Every name listed
+ * above must appear exactly once.  Synchronous; the caller keeps ownership
+ * of the inputs and may free them on return. */
+rtv_status rtv_load_expert(rtv_ctx* ctx, const rtv_tensor* params, int n_params);
+
+/* Install the prefix KV cache ([DM0.5] 5.1): `kv` is a device or host array
+ * [n_layers][2][batch][prefix_len][n_kv_heads][head_dim] in the config dtype
+ * (index 0 = keys, already rotated; 1 = values).  It is copied on `stream`
+ * into library-owned memory of fixed address (the static-address contract
+ * of [DM0.5] 6.5).  prefix_len <= max_prefix_len, batch <= max_batch. */
+rtv_status rtv_set_prefix_kv(rtv_ctx* ctx, const void* kv, int prefix_len, int batch, rtv_stream stream);
+
+/* Denoise ([DM0.5] 5.3): from noise x_1 = noise [batch][H][A], run n_steps
+ * Euler steps x <- x - (1/n_steps) * v(x, t_k), t_k = 1 - k/n_steps, and
+ * write the action chunk [batch][H][A] to actions_out.  state is
+ * [batch][Sd].  batch is the one given to rtv_set_prefix_kv.  Each pointer
+ * may be device or host memory (host copies are enqueued on `stream`).
+ * The first call for a given (n_steps, batch, prefix_len) captures a CUDA
+ * graph (not on `stream`); later calls replay it. */
+rtv_status rtv_denoise(rtv_ctx* ctx, const float* noise, const float* state, int n_steps,
+                       float* actions_out, rtv_stream stream);
+
+/* FLASH verification ([FLASH] 02, 03.2, 03.3) of one draft chunk against
+ * the prefix of batch element 0: for each tau_i (host array of n_taus
+ * values in [0,1]) form X_i = tau_i*noise + (1-tau_i)*draft, evaluate the
+ * expert once on all X_i together (each sees the prefix and its own
+ * suffix), rebuild A_i = X_i - tau_i*v_i, take d_i[h] = ||A_i[h] - draft[h]||_2
+ * and accept the longest prefix with d_i[h] < delta for every i.
+ * draft, noise [H][A], state [Sd]: device or host.  Outputs (device or
+ * host): *accepted_len (int32), *flags (RTV_FLAG_*), dist [n_taus][H] fp32
+ * or NULL.  gripper_dim in [0, A) selects the gripper action dimension. */
+rtv_status rtv_verify(rtv_ctx* ctx, const float* draft, const float* noise, const float* state,
+                      const float* taus, int n_taus, float delta, int gripper_dim,
+                      int* accepted_len, unsigned* flags, float* dist, rtv_stream stream);
+
+/* Synchronise the context's device work and report the device status word
+ * (RTV_DEV_* bits); the word is cleared after it is read.  Returns
+ * RTV_ERR_TIMEOUT / RTV_ERR_NUMERIC when the matching bit was set. */
+rtv_status rtv_device_status(rtv_ctx* ctx, unsigned* bits);
+
+/* Last error message of the context (never NULL; "" when none). */
+const char* rtv_last_error(rtv_ctx* ctx);
+
+/* Human-readable name of the kernel path a context uses ("tcgen05", "simt"). */
+const char* rtv_path_name(rtv_ctx* ctx);
+
+/* Number of kernel launches one call makes: of the graph captured for
+ * rtv_denoise(n_steps = n, current prefix batch) when is_verify = 0, or of
+ * rtv_verify(n_taus = n) when is_verify = 1.  -1 if that graph has not been
+ * captured yet.  Diagnostic; enqueues nothing. */
+int rtv_graph_kernel_count(rtv_ctx* ctx, int n, int is_verify);
+
+/* Release every resource of the context.  NULL is accepted. */
+void rtv_destroy(rtv_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RTV_H */
