@@ -15,11 +15,17 @@ rtv_status fast_create(rtv_ctx* ctx);
 // Pack the loaded parameters into the tensor-core layouts.
 rtv_status fast_load(rtv_ctx* ctx, const rtv_tensor* params, int n_params);
 bool fast_supports_prefix(rtv_ctx* ctx, int prefix_len);
-// Expert forward over G suffixes into ctx->h (same contract as the SIMT forward).
-rtv_status fast_expert(rtv_ctx* ctx, int G, int P, const float* c, int c_stride, int state_stride,
-                       int prefix_batch_stride, const float* rope_cs, const float* rope_sn, cudaStream_t st);
-// Output head: Euler step on ctx->x (velocity_only = false) or v into ctx->v.
-void fast_out_head(rtv_ctx* ctx, int G, float dt, bool velocity_only, cudaStream_t st);
+// Step boundary over G suffixes: output head (Euler update of ctx->x, or the
+// velocity into ctx->v when velocity_only) and/or the suffix embedding of the
+// next evaluation into ctx->h with time condition rows c (stride c_stride).
+rtv_status fast_step(rtv_ctx* ctx, int G, bool do_head, bool do_embed, float dt, const float* c, int c_stride,
+                     int state_stride, bool velocity_only, cudaStream_t st);
+// The expert's layers over G suffixes (residual stream ctx->h).
+rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, const float* rope_cs,
+                       const float* rope_sn, cudaStream_t st);
 void fast_destroy(rtv_ctx* ctx);
+// Diagnostic phase trace (only when the RTV_TRACE environment variable is set).
+void fast_arm_trace(rtv_ctx* ctx);
+void fast_trace_report(rtv_ctx* ctx);
 
 }  // namespace rtv

@@ -97,21 +97,28 @@ __global__ void embed_kernel(const float* __restrict__ x, const float* __restric
                              const WT* __restrict__ w_sp, const float* __restrict__ b_sp, const WT* __restrict__ w_ai,
                              const float* __restrict__ b_ai, const float* __restrict__ c, int c_group_stride,
                              float* __restrict__ h, int w, int S, int A, int Sd) {
+  __shared__ float xin[64];
   const int r = blockIdx.x;
   const int g = r / S, s = r % S;
+  const float* src = s == 0 ? state + (size_t)g * state_group_stride : x + ((size_t)g * (S - 1) + (s - 1)) * A;
+  const int K = s == 0 ? Sd : A;
+  const WT* W = s == 0 ? w_sp : w_ai;
   for (int i = threadIdx.x; i < w; i += blockDim.x) {
-    float acc;
-    if (s == 0) {
-      const float* st = state + (size_t)g * state_group_stride;
-      acc = 0.f;
-      for (int k = 0; k < Sd; ++k) acc = fmaf(to_f32(w_sp[(size_t)i * Sd + k]), st[k], acc);
-      acc += b_sp[i];
-    } else {
-      const float* xr = x + ((size_t)g * (S - 1) + (s - 1)) * A;
-      acc = 0.f;
-      for (int k = 0; k < A; ++k) acc = fmaf(to_f32(w_ai[(size_t)i * A + k]), xr[k], acc);
-      acc = acc + b_ai[i] + c[(size_t)g * c_group_stride + i];
+    float acc = 0.f;
+    for (int k0 = 0; k0 < K; k0 += 64) {
+      __syncthreads();
+      for (int kk = threadIdx.x; kk < 64; kk += blockDim.x) xin[kk] = (k0 + kk < K) ? src[k0 + kk] : 0.f;
+      __syncthreads();
+      // all weight loads of the chunk are independent: issue them together
+      float wv[64];
+#pragma unroll
+      for (int k = 0; k < 64; ++k) wv[k] = (k0 + k < K) ? to_f32(W[(size_t)i * K + k0 + k]) : 0.f;
+#pragma unroll
+      for (int k = 0; k < 64; ++k)
+        if (k0 + k < K) acc = fmaf(wv[k], xin[k], acc);
     }
+    acc += s == 0 ? b_sp[i] : b_ai[i];
+    if (s != 0) acc += c[(size_t)g * c_group_stride + i];
     h[(size_t)r * w + i] = acc;
   }
 }
@@ -269,17 +276,37 @@ __global__ void out_head_kernel(const float* __restrict__ h, const float* __rest
   const int g = blockIdx.x / H, j = blockIdx.x % H;
   const float* row = h + ((size_t)g * S + 1 + j) * w;
   float ss = 0.f;
-  for (int i = threadIdx.x; i < w; i += blockDim.x) ss = fmaf(row[i], row[i], ss);
+  for (int i = threadIdx.x; i < w; i += blockDim.x) {
+    const float v = row[i];
+    hn[i] = v;
+    ss = fmaf(v, v, ss);
+  }
   ss = block_sum(ss, red);
   const float inv = rsqrtf(ss / (float)w + eps);
-  for (int i = threadIdx.x; i < w; i += blockDim.x) hn[i] = row[i] * inv * (1.f + gain[i]);
+  for (int i = threadIdx.x; i < w; i += blockDim.x) hn[i] = hn[i] * inv * (1.f + gain[i]);
   __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  for (int a = warp; a < A; a += nw) {
+  // 8 threads per output: each takes w/8 consecutive inputs (loads issued together)
+  const int sub = threadIdx.x & 7;
+  const int per = w / 8;
+  for (int a0 = threadIdx.x >> 3; a0 < ((A + 31) / 32) * 32; a0 += blockDim.x >> 3) {
+    const int a = a0;
     float dot = 0.f;
-    for (int i = lane; i < w; i += 32) dot = fmaf(to_f32(w_ao[(size_t)a * w + i]), hn[i], dot);
-    dot = warp_sum(dot);
-    if (lane == 0) {
+    if (a < A) {
+      const WT* wr = w_ao + (size_t)a * w + sub * per;
+      const float* hr = hn + sub * per;
+      for (int i0 = 0; i0 < per; i0 += 32) {
+        float wv[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) wv[i] = (i0 + i < per) ? to_f32(wr[i0 + i]) : 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (i0 + i < per) dot = fmaf(wv[i], hr[i0 + i], dot);
+      }
+    }
+    dot += __shfl_xor_sync(0xffffffffu, dot, 4);
+    dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+    dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+    if (sub == 0 && a < A) {
       const float v = dot + b_ao[a];
       const size_t off = ((size_t)g * H + j) * A + a;
       if (vout) {
@@ -393,8 +420,9 @@ template <typename WT>
 void launch_embed(const float* x, const float* state, int state_group_stride, const WT* w_sp, const float* b_sp,
                   const WT* w_ai, const float* b_ai, const float* c, int c_group_stride, float* h, int G, int w,
                   int S, int A, int Sd, cudaStream_t st) {
-  embed_kernel<WT><<<G * S, 256, 0, st>>>(x, state, state_group_stride, w_sp, b_sp, w_ai, b_ai, c, c_group_stride, h,
-                                          w, S, A, Sd);
+  const int threads = (w % 256 == 0) ? 256 : (w % 128 == 0 ? 128 : (w % 64 == 0 ? 64 : 32));
+  embed_kernel<WT><<<G * S, threads, 0, st>>>(x, state, state_group_stride, w_sp, b_sp, w_ai, b_ai, c, c_group_stride,
+                                              h, w, S, A, Sd);
 }
 template void launch_embed<float>(const float*, const float*, int, const float*, const float*, const float*,
                                   const float*, const float*, int, float*, int, int, int, int, int, cudaStream_t);

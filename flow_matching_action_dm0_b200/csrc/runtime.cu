@@ -148,25 +148,38 @@ rtv_status build_graph(rtv_ctx* ctx, int kind, int n, int batch, int P, GraphEnt
   CK(cudaGetLastError());
   CK(cudaStreamSynchronize(st));
 
+  if (ctx->use_fast) fast_arm_trace(ctx);
   CK(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
-  bool fast = ctx->use_fast;
   rtv_status fs = RTV_OK;
+  auto chain = [&](rtv_status s2) {
+    if (fs == RTV_OK) fs = s2;
+  };
   if (kind == KIND_DENOISE) {
     const float dt = (float)(1.0 / (double)n);
-    for (int step = 0; step < n && fs == RTV_OK; ++step) {
-      if (fast) fs = fast_expert(ctx, batch, P, ctab + (size_t)step * w, 0, k.state_dim, 1, cs, sn, st);
-      else simt_expert<WT>(ctx, batch, P, ctab + (size_t)step * w, 0, k.state_dim, 1, cs, sn, st);
-      if (fast) fast_out_head(ctx, batch, dt, false, st);
-      else launch_out_head<WT>(ctx->h, ctx->W.g_final, (const WT*)ctx->W.ao_w, ctx->W.ao_b, ctx->x, nullptr, dt,
-                               batch, w, S, k.action_dim, k.rms_eps, ctx->status, st);
+    if (ctx->use_fast) {
+      // step boundary k: head of step k-1 (k > 0) and embedding of step k (k < n)
+      chain(fast_step(ctx, batch, false, true, dt, ctab, 0, k.state_dim, false, st));
+      for (int step = 0; step < n && fs == RTV_OK; ++step) {
+        chain(fast_layers(ctx, batch, P, 1, cs, sn, st));
+        const bool more = step + 1 < n;
+        chain(fast_step(ctx, batch, true, more, dt, more ? ctab + (size_t)(step + 1) * w : ctab, 0, k.state_dim,
+                        false, st));
+      }
+    } else {
+      for (int step = 0; step < n; ++step) {
+        simt_expert<WT>(ctx, batch, P, ctab + (size_t)step * w, 0, k.state_dim, 1, cs, sn, st);
+        launch_out_head<WT>(ctx->h, ctx->W.g_final, (const WT*)ctx->W.ao_w, ctx->W.ao_b, ctx->x, nullptr, dt, batch,
+                            w, S, k.action_dim, k.rms_eps, ctx->status, st);
+      }
     }
   } else {
     const int T = n;
     launch_verify_interp(ctx->draft, ctx->eps, ctx->taus, ctx->x, T, ctx->H * k.action_dim, st);
     time_condition<WT>(ctx, ctx->taus, T, 0, ctx->c_verify, st);
-    if (fast) {
-      fs = fast_expert(ctx, T, P, ctx->c_verify, w, 0, 0, cs, sn, st);
-      fast_out_head(ctx, T, 0.f, true, st);
+    if (ctx->use_fast) {
+      chain(fast_step(ctx, T, false, true, 0.f, ctx->c_verify, w, 0, false, st));
+      chain(fast_layers(ctx, T, P, 0, cs, sn, st));
+      chain(fast_step(ctx, T, true, false, 0.f, ctx->c_verify, w, 0, true, st));
     } else {
       simt_expert<WT>(ctx, T, P, ctx->c_verify, w, 0, 0, cs, sn, st);
       launch_out_head<WT>(ctx->h, ctx->W.g_final, (const WT*)ctx->W.ao_w, ctx->W.ao_b, ctx->x, ctx->v, 0.f, T, w,
@@ -242,7 +255,7 @@ rtv_status rtv_create(const rtv_expert_config* cfg_in, int cuda_device, rtv_ctx*
   if (k.n_layers <= 0 || k.width <= 0 || k.width % 2 || k.n_q_heads <= 0 || k.n_kv_heads <= 0 ||
       k.n_q_heads % k.n_kv_heads || k.head_dim <= 0 || k.head_dim % 2 || k.mlp_dim <= 0 || k.action_dim <= 0 ||
       k.state_dim <= 0 || k.chunk_len <= 0 || k.max_prefix_len <= 0 || k.max_batch <= 0 || k.max_taus < 0 ||
-      k.width < 4)
+      k.width < 32 || k.width % 32)
     return RTV_ERR_ARG;
   if (k.dtype != RTV_F32 && k.dtype != RTV_BF16) return RTV_ERR_ARG;
   if (k.mlp_dtype == RTV_SAME) k.mlp_dtype = k.dtype;
@@ -456,6 +469,7 @@ rtv_status rtv_denoise(rtv_ctx* ctx, const float* noise, const float* state, int
   CK(cudaMemcpyAsync(ctx->state, state, (size_t)B * k.state_dim * sizeof(float), cudaMemcpyDefault, st));
   CK(cudaGraphLaunch(ge->exec, st));
   CK(cudaMemcpyAsync(actions_out, ctx->x, xb, cudaMemcpyDefault, st));
+  if (ctx->use_fast && getenv("RTV_TRACE")) fast_trace_report(ctx);
   return RTV_OK;
 }
 
