@@ -72,17 +72,20 @@ struct GemmArgs {
 };
 
 // Phase stamps of the optional trace (one row of 16 per CTA).
-enum { TR_START = 0, TR_W_ISSUED, TR_PDL, TR_FIRST_FULL, TR_MMA_ISSUED, TR_DONE, TR_COPIED, TR_RECV, TR_END };
+enum { TR_START = 0, TR_W_ISSUED, TR_PDL, TR_FIRST_FULL, TR_MMA_ISSUED, TR_DONE, TR_COPIED, TR_RECV, TR_END,
+       TR_PREFETCHED, TR_ARRIVED, TR_ITER0, TR_EXIT };
 
 struct GemmSmem {
-  int stages, stage_bytes, ring_bytes, part_off, recv_off, bar_off, total;
+  int stages, stage_bytes, ring_bytes, part_off, recv_off, in_off, bar_off, total;
 };
 
 // Shared memory of one GEMM CTA: a ring of `stages` stages, each a 128x64
 // bf16 weight box (16 KB) and the matching 64-wide bf16 activation box of
 // n_mma token rows, both K-major with the 128-byte swizzle; the fp32 partial
 // tile [n_mma][128] (over the ring once the MMAs are done, when it fits);
-// the receive buffer [cs * per][128] of the cluster reduction; mbarriers.
+// the receive buffer [cs * per][128] of the cluster reduction; the
+// epilogue's per-token inputs [per][128] (residual rows or RoPE cos/sin);
+// mbarriers.
 __host__ __device__ inline GemmSmem gemm_smem_layout(int stages, int n_mma, int cs, int T) {
   GemmSmem s;
   const int per = (T + cs - 1) / cs;
@@ -92,7 +95,8 @@ __host__ __device__ inline GemmSmem gemm_smem_layout(int stages, int n_mma, int 
   const int part_bytes = n_mma * 512;
   s.part_off = part_bytes <= s.ring_bytes ? 0 : s.ring_bytes;
   s.recv_off = s.ring_bytes > s.part_off + part_bytes ? s.ring_bytes : s.part_off + part_bytes;
-  s.bar_off = s.recv_off + cs * per * 512;
+  s.in_off = s.recv_off + cs * per * 512;   // [per][128] fp32 epilogue inputs of the owned tokens
+  s.bar_off = s.in_off + per * 512;
   s.total = s.bar_off + (2 * stages + 2) * 8 + 16 + 1024;   // barriers, TMEM slot, alignment slack
   return s;
 }
@@ -135,13 +139,13 @@ template <int MODE>
 __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap wmap,
                                                          const __grid_constant__ CUtensorMap amap, const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ float sq_x[4];
+  __shared__ float rs_s[64];
   const int n_mma = a.n_mma;
   const int cs = gridDim.x;
   const GemmSmem L = gemm_smem_layout(a.stages, n_mma, cs, a.T);
   // every CTA of the grid sees the same values, so a refusal is uniform across each cluster
   if (dynamic_smem_size() < (uint32_t)L.total || a.kslice < 64 || (a.kslice & 63) || a.stages < 1 || n_mma > 256 ||
-      (n_mma & 15) || a.T > n_mma || cs > 16) {
+      (n_mma & 15) || a.T > n_mma || cs > 16 || (a.T + cs - 1) / cs > 64) {
     if (threadIdx.x == 0) atomicOr(a.status, RTV_DEV_BOUNDS);
     return;
   }
@@ -262,11 +266,17 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     // accumulator -> this CTA's partial tile [token][feature]
     const int quarter = warp & 3;
     const int f = quarter * 32 + lane;
-    for (int c = 0; c < n_mma; c += 16) {
-      float v[16];
-      ptx::tmem_ld_16(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c, v);
+    for (int c = 0; c < n_mma; c += 32) {
+      float v[32];
+      if (c + 16 < n_mma) {
+        ptx::tmem_ld_32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c, v);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) part[(c + i) * 128 + f] = v[i];
+        for (int i = 0; i < 32; ++i) part[(c + i) * 128 + f] = v[i];
+      } else {
+        ptx::tmem_ld_16(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c, *reinterpret_cast<float(*)[16]>(v));
+#pragma unroll
+        for (int i = 0; i < 16; ++i) part[(c + i) * 128 + f] = v[i];
+      }
     }
     ptx::tc_fence_before();
     ptx::fence_proxy_async_smem();
@@ -282,75 +292,112 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       }
       if (trace) trace[TR_COPIED] = ptx::globaltimer();
     }
+    // Everything the epilogue reads from global memory is requested now, in
+    // parallel, while the partials are still in flight: the owned tokens'
+    // residual rows of this tile (O, DOWN) or their RoPE cos/sin (QKV) go to
+    // shared memory by cp.async; 1/rms of the owned tokens (QKV, GU) too.
+    float* in_s = (float*)(base + L.in_off);
+    const int n_wt = a.w >> 7;
+    const int tph = a.D >> 7, hd = a.D >> 1;
+    const int hh = nt / tph, dq0 = 64 * (nt - (nt / tph) * tph);
+    const bool rope = MODE == GM_QKV && hh < a.Hq + a.Hkv;
+    const uint32_t in_a = ptx::smem_u32(in_s);
+    if (MODE == GM_O || MODE == GM_DOWN) {
+      for (int c = tid; c < n_own * 32; c += 128) {
+        const int tl = c >> 5, ch = c & 31;
+        ptx::cp_async_16(in_a + (uint32_t)(c * 16), a.h + (size_t)(t_own0 + tl) * a.w + nt * 128 + ch * 4);
+      }
+    } else if (rope) {
+      for (int c = tid; c < n_own * 32; c += 128) {
+        const int tl = c >> 5, ch = c & 31;   // chunks 0-15: cos, 16-31: sin (64 floats each)
+        const int s = (t_own0 + tl) % a.S;
+        const float* src = (ch < 16 ? a.rope_cs : a.rope_sn) + (size_t)s * hd + dq0 + (ch & 15) * 4;
+        ptx::cp_async_16(in_a + (uint32_t)(c * 16), src);
+      }
+    }
+    if ((MODE == GM_QKV || MODE == GM_GU) && tid < n_own) {
+      float sst = 0.f;
+      for (int j2 = 0; j2 < n_wt; ++j2) sst += a.ssp[(size_t)(t_own0 + tid) * n_wt + j2];
+      rs_s[tid] = rsqrtf(sst / (float)a.w + a.eps);
+    }
+    ptx::cp_async_wait_all();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (trace && tid == 0) trace[TR_PREFETCHED] = ptx::globaltimer();
     if (!ptx::mbar_wait(rbar, 0, a.timeout_ns)) atomicOr(a.status, RTV_DEV_TIMEOUT);
     if (trace && tid == 0) trace[TR_RECV] = ptx::globaltimer();
     cluster_arrive_release();   // my incoming copies are complete
+    if (trace && tid == 0) trace[TR_ARRIVED] = ptx::globaltimer();
 
     // ---- reduction in rank order + epilogue for the tokens this rank owns ----
-    const int p = tid & 63, half = tid >> 6;
-    const int n_wt = a.w >> 7;
-    for (int tl = half; tl < ((n_own + 1) & ~1); tl += 2) {
-      const bool valid = tl < n_own;
+    // one warp per token; lane l takes features (2l, 2l+1) and (2l+64, 2l+65)
+    const int ew = warp - 2;
+    const int f0 = 2 * lane;
+    const int n1 = nt * 128 + f0, n2 = n1 + 64;
+    float2 gn1 = make_float2(0.f, 0.f), gn2 = make_float2(0.f, 0.f);
+    if ((MODE == GM_O || MODE == GM_DOWN) && a.g_next) {
+      gn1 = *reinterpret_cast<const float2*>(a.g_next + n1);
+      gn2 = *reinterpret_cast<const float2*>(a.g_next + n2);
+    }
+#pragma unroll 1
+    for (int tl = ew; tl < n_own; tl += 4) {
       const int t = t_own0 + tl;
-      float x1 = 0.f, x2 = 0.f;
-      if (valid) {
-        for (int qr = 0; qr < cs; ++qr) {
-          const float* rr = recv + (qr * per + tl) * 128;
-          x1 += rr[p];
-          x2 += rr[p + 64];
-        }
+      float2 x1 = make_float2(0.f, 0.f), x2 = make_float2(0.f, 0.f);
+      for (int qr = 0; qr < cs; ++qr) {
+        const float* rr = recv + (qr * per + tl) * 128;
+        const float2 u1 = *reinterpret_cast<const float2*>(rr + f0);
+        const float2 u2 = *reinterpret_cast<const float2*>(rr + 64 + f0);
+        x1.x += u1.x;
+        x1.y += u1.y;
+        x2.x += u2.x;
+        x2.y += u2.y;
       }
       if (MODE == GM_O || MODE == GM_DOWN) {
         // residual add, then the next norm's bf16 input and this tile's sum of squares
-        const int n1 = nt * 128 + p, n2 = n1 + 64;
-        float h1 = 0.f, h2 = 0.f;
-        if (valid) {
-          float* hr = a.h + (size_t)t * a.w;
-          h1 = hr[n1] + x1;
-          h2 = hr[n2] + x2;
-          hr[n1] = h1;
-          hr[n2] = h2;
-        }
+        const float2 r1 = *reinterpret_cast<const float2*>(in_s + tl * 128 + f0);
+        const float2 r2 = *reinterpret_cast<const float2*>(in_s + tl * 128 + 64 + f0);
+        const float2 h1 = make_float2(r1.x + x1.x, r1.y + x1.y);
+        const float2 h2 = make_float2(r2.x + x2.x, r2.y + x2.y);
+        *reinterpret_cast<float2*>(a.h + (size_t)t * a.w + n1) = h1;
+        *reinterpret_cast<float2*>(a.h + (size_t)t * a.w + n2) = h2;
         if (a.g_next) {
-          float sq = fmaf(h1, h1, h2 * h2);
+          float sq = h1.x * h1.x;
+          sq = fmaf(h1.y, h1.y, sq);
+          sq = fmaf(h2.x, h2.x, sq);
+          sq = fmaf(h2.y, h2.y, sq);
           sq = warp_sum(sq);
-          // two warps per token: combine their sums in a fixed order
-          if (lane == 0) sq_x[warp - 2] = sq;
-          asm volatile("bar.sync %0, 64;" ::"r"(3 + half) : "memory");
-          if (valid) {
-            a.hb[(size_t)t * a.w + n1] = __float2bfloat16_rn(h1 * (1.f + a.g_next[n1]));
-            a.hb[(size_t)t * a.w + n2] = __float2bfloat16_rn(h2 * (1.f + a.g_next[n2]));
-            if (p == 0) a.ssp[(size_t)t * n_wt + nt] = sq_x[2 * half] + sq_x[2 * half + 1];
-          }
-          asm volatile("bar.sync %0, 64;" ::"r"(3 + half) : "memory");
+          *reinterpret_cast<uint32_t*>(a.hb + (size_t)t * a.w + n1) =
+              ptx::pack_bf16x2(h1.x * (1.f + gn1.x), h1.y * (1.f + gn1.y));
+          *reinterpret_cast<uint32_t*>(a.hb + (size_t)t * a.w + n2) =
+              ptx::pack_bf16x2(h2.x * (1.f + gn2.x), h2.y * (1.f + gn2.y));
+          if (lane == 0) a.ssp[(size_t)t * n_wt + nt] = sq;
         }
-      } else if (valid) {
-        float sst = 0.f;
-        for (int j2 = 0; j2 < n_wt; ++j2) sst += a.ssp[(size_t)t * n_wt + j2];
-        const float rs = rsqrtf(sst / (float)a.w + a.eps);
-        x1 *= rs;
-        x2 *= rs;
+      } else {
+        const float rs = rs_s[tl];
+        x1.x *= rs;
+        x1.y *= rs;
+        x2.x *= rs;
+        x2.y *= rs;
         if (MODE == GM_GU) {
-          a.m[(size_t)t * a.F + nt * 64 + p] = __float2bfloat16_rn(gelu_tanh(x1) * x2);
+          *reinterpret_cast<uint32_t*>(a.m + (size_t)t * a.F + nt * 64 + f0) =
+              ptx::pack_bf16x2(gelu_tanh(x1.x) * x2.x, gelu_tanh(x1.y) * x2.y);
         } else {
-          const int tph = a.D >> 7;
-          const int hh = nt / tph, bq = nt - hh * tph;
-          const int d = 64 * bq + p, hd = a.D >> 1;
           const int g = t / a.S, s = t - g * a.S;
-          float y1 = x1, y2 = x2;
-          if (hh < a.Hq + a.Hkv) {
-            const float c = a.rope_cs[s * hd + d], sn = a.rope_sn[s * hd + d];
-            y1 = x1 * c - x2 * sn;
-            y2 = x2 * c + x1 * sn;
+          float2 y1 = x1, y2 = x2;
+          if (rope) {
+            const float2 c = *reinterpret_cast<const float2*>(in_s + tl * 128 + f0);
+            const float2 sn = *reinterpret_cast<const float2*>(in_s + tl * 128 + 64 + f0);
+            y1 = make_float2(x1.x * c.x - x2.x * sn.x, x1.y * c.y - x2.y * sn.y);
+            y2 = make_float2(x2.x * c.x + x1.x * sn.x, x2.y * c.y + x1.y * sn.y);
           }
           __nv_bfloat16* dst;
           if (hh < a.Hq) dst = a.q + ((size_t)t * a.Hq + hh) * a.D;
           else if (hh < a.Hq + a.Hkv) dst = a.ks + (((size_t)g * a.Hkv + (hh - a.Hq)) * a.S + s) * a.D;
           else dst = a.vs + (((size_t)g * a.Hkv + (hh - a.Hq - a.Hkv)) * a.S + s) * a.D;
-          dst[d] = __float2bfloat16_rn(y1);
-          dst[d + hd] = __float2bfloat16_rn(y2);
+          *reinterpret_cast<uint32_t*>(dst + dq0 + f0) = ptx::pack_bf16x2(y1.x, y1.y);
+          *reinterpret_cast<uint32_t*>(dst + dq0 + f0 + hd) = ptx::pack_bf16x2(y2.x, y2.y);
         }
       }
+      if (trace && tid == 0 && tl == 0) trace[TR_ITER0] = ptx::globaltimer();
     }
     if (trace && tid == 0) trace[TR_END] = ptx::globaltimer();
   }
@@ -359,6 +406,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     cluster_arrive_release();   // nothing incoming to wait for
   }
   cluster_wait();   // every rank's incoming copies are complete: no copy still reads my shared memory
+  if (trace && threadIdx.x == 64) trace[TR_EXIT] = ptx::globaltimer();
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, ncols);
@@ -388,13 +436,15 @@ struct AttnArgs {
   const __nv_bfloat16* sv;
   __nv_bfloat16* o;          // [T][Hq*D]
   unsigned* status;
+  unsigned long long* trace; // optional phase stamps [cta][16], or nullptr
   int S, P, Pmax, Hq, Hkv, pbs, mask_mode, kpc;
   float scale_log2;
 };
 
-// Q tile, K and V tiles, receive buffers of the cluster combine, combine weights.
+// Q tile, K and V tiles, receive buffers of the cluster combine (bf16 rows +
+// fp32 max/sum), combine weights.
 __host__ __device__ inline int attn_smem_bytes(int D, int nchunk, int rpc) {
-  return 64 * D * 2 + 2 * 128 * D * 2 + nchunk * rpc * (D + 2) * 4 + rpc * (nchunk + 1) * 4;
+  return 64 * D * 2 + 2 * 128 * D * 2 + nchunk * rpc * D * 2 + nchunk * rpc * 2 * 4 + rpc * (nchunk + 1) * 4;
 }
 
 template <int D>
@@ -410,8 +460,8 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const AttnArgs a) {
   __nv_bfloat16* Qs = reinterpret_cast<__nv_bfloat16*>(sm_attn);
   __nv_bfloat16* Ks = Qs + 64 * D;
   __nv_bfloat16* Vs = Ks + 128 * D;
-  float* recv = reinterpret_cast<float*>(Vs + 128 * D);   // [nchunk][rpc][D] partial outputs pushed to me
-  float* recv_ml = recv + nchunk * rpc * D;                // [nchunk][rpc][2] (running max, sum)
+  __nv_bfloat16* recv = Vs + 128 * D;                      // [nchunk][rpc][D] partial outputs pushed to me
+  float* recv_ml = reinterpret_cast<float*>(recv + nchunk * rpc * D);   // [nchunk][rpc][2] (running max, sum)
   float* wq_s = recv_ml + nchunk * rpc * 2;                 // [rpc][nchunk] combine weights
   float* inv_s = wq_s + rpc * nchunk;                       // [rpc] 1 / combined sum
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -428,9 +478,13 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const AttnArgs a) {
   const __nv_bfloat16* skh = a.sk + ((size_t)g * a.Hkv + kvh) * a.S * D;
   const __nv_bfloat16* svh = a.sv + ((size_t)g * a.Hkv + kvh) * a.S * D;
 
+  unsigned long long* trace =
+      a.trace ? a.trace + (((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * 16 : nullptr;
+  if (trace && tid == 0) trace[0] = ptx::globaltimer();
   cluster_arrive_relaxed();
   ptx::pdl_launch_dependents();
   ptx::pdl_wait();
+  if (trace && tid == 0) trace[1] = ptx::globaltimer();
 
   const uint32_t qs_a = ptx::smem_u32(Qs), ks_a = ptx::smem_u32(Ks), vs_a = ptx::smem_u32(Vs);
   for (int c = tid; c < 64 * CPR; c += 256) {
@@ -464,6 +518,7 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const AttnArgs a) {
     }
     ptx::cp_async_wait_all();
     __syncthreads();
+    if (trace && tid == 0 && kt == kb) trace[2] = ptx::globaltimer();
     const int kbase = 64 * kh;   // this warp's half of the tile
     if (kt + kbase < ke) {
       // scores S = Q K^T for this warp's 16 rows x 64 keys
@@ -548,6 +603,7 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const AttnArgs a) {
     }
   }
   ptx::cp_async_wait_all();
+  if (trace && tid == 0) trace[3] = ptx::globaltimer();
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     l_r[i] += __shfl_xor_sync(0xffffffffu, l_r[i], 1);
@@ -555,14 +611,19 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const AttnArgs a) {
   }
   // merge the two key halves of each row block in shared memory (K/V tiles are dead)
   __syncthreads();
-  float* xo = reinterpret_cast<float*>(Ks);        // [64 rows][D] fp32 = exactly the K tile's bytes
-  float* xml = reinterpret_cast<float*>(Vs);       // [64 rows][2]
+  // padded row strides keep the fragment-order accesses below free of bank conflicts
+  constexpr int XS = D + 8;                                      // fp32 row stride of xo
+  constexpr int OS = D + 8;                                      // bf16 row stride of ob_s
+  float* xo = reinterpret_cast<float*>(Ks);                      // [64 rows][XS] fp32   (K and V tiles are dead)
+  __nv_bfloat16* ob_s = reinterpret_cast<__nv_bfloat16*>(xo + 64 * XS);   // [64 rows][OS] merged rows, bf16
+  float* xml = reinterpret_cast<float*>(Qs);                     // [64 rows][2] (the Q tile is dead too)
+  float* mml = reinterpret_cast<float*>(Qs) + 64 * 2;            // [64 rows][2] merged (max, sum)
   if (kh == 1) {
 #pragma unroll
     for (int nt = 0; nt < D / 8; ++nt) {
       const int d = 8 * nt + 2 * (lane & 3);
-      *reinterpret_cast<float2*>(xo + row0 * D + d) = make_float2(o_acc[nt][0], o_acc[nt][1]);
-      *reinterpret_cast<float2*>(xo + (row0 + 8) * D + d) = make_float2(o_acc[nt][2], o_acc[nt][3]);
+      *reinterpret_cast<float2*>(xo + row0 * XS + d) = make_float2(o_acc[nt][0], o_acc[nt][1]);
+      *reinterpret_cast<float2*>(xo + (row0 + 8) * XS + d) = make_float2(o_acc[nt][2], o_acc[nt][3]);
     }
     if ((lane & 3) == 0) {
       xml[row0 * 2] = m_r[0];
@@ -572,8 +633,6 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const AttnArgs a) {
     }
   }
   __syncthreads();
-  cluster_wait();   // entry phase: every rank has started
-  const uint32_t rcv = ptx::smem_u32(recv), rml = ptx::smem_u32(recv_ml);
   if (kh == 0) {
 #pragma unroll
     for (int hrow = 0; hrow < 2; ++hrow) {
@@ -582,27 +641,47 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const AttnArgs a) {
       const float mm = fmaxf(m_r[hrow], m2);
       const float w1 = m_r[hrow] == -INFINITY ? 0.f : exp2f(m_r[hrow] - mm);
       const float w2 = m2 == -INFINITY ? 0.f : exp2f(m2 - mm);
-      const float ll = l_r[hrow] * w1 + l2 * w2;
-      if (r < a.S) {
-        const int owner = r / rpc, rl = r - owner * rpc;
-        const uint32_t dst = ptx::mapa(rcv, (uint32_t)owner) + (uint32_t)(((rank * rpc + rl) * D) * 4);
 #pragma unroll
-        for (int nt = 0; nt < D / 8; ++nt) {
-          const int d = 8 * nt + 2 * (lane & 3);
-          const float2 o2 = *reinterpret_cast<const float2*>(xo + r * D + d);
-          const float vx = o_acc[nt][2 * hrow] * w1 + o2.x * w2;
-          const float vy = o_acc[nt][2 * hrow + 1] * w1 + o2.y * w2;
-          asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(dst + (uint32_t)(d * 4)), "f"(vx), "f"(vy)
-                       : "memory");
-        }
-        if ((lane & 3) == 0) {
-          const uint32_t mdst = ptx::mapa(rml, (uint32_t)owner) + (uint32_t)((rank * rpc + rl) * 8);
-          asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(mdst), "f"(mm), "f"(ll) : "memory");
-        }
+      for (int nt = 0; nt < D / 8; ++nt) {
+        const int d = 8 * nt + 2 * (lane & 3);
+        const float2 o2 = *reinterpret_cast<const float2*>(xo + r * XS + d);
+        *reinterpret_cast<uint32_t*>(ob_s + r * OS + d) =
+            ptx::pack_bf16x2(o_acc[nt][2 * hrow] * w1 + o2.x * w2, o_acc[nt][2 * hrow + 1] * w1 + o2.y * w2);
+      }
+      if ((lane & 3) == 0) {
+        mml[r * 2] = mm;
+        mml[r * 2 + 1] = l_r[hrow] * w1 + l2 * w2;
       }
     }
   }
+  __syncthreads();
+  if (trace && tid == 0) trace[4] = ptx::globaltimer();
+  cluster_wait();   // entry phase: every rank has started
+  if (trace && tid == 0) trace[5] = ptx::globaltimer();
+  // push every valid row (D bf16 = D*2 bytes) to the rank that combines it:
+  // one warp per row, 16 bytes per lane
+  {
+    const uint32_t rcv = ptx::smem_u32(recv), rml = ptx::smem_u32(recv_ml);
+    constexpr int CPRB = D / 8;   // 16-byte chunks per bf16 row
+    for (int r = warp; r < a.S; r += 8) {
+      const int owner = r / rpc, rl = r - owner * rpc;
+      const uint32_t dst = ptx::mapa(rcv, (uint32_t)owner) + (uint32_t)((rank * rpc + rl) * D * 2);
+      for (int ch = lane; ch < CPRB; ch += 32) {
+        const uint4 v = *reinterpret_cast<const uint4*>(ob_s + r * OS + ch * 8);
+        asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + (uint32_t)(ch * 16)), "r"(v.x),
+                     "r"(v.y), "r"(v.z), "r"(v.w)
+                     : "memory");
+      }
+      if (lane == 0) {
+        const uint32_t mdst = ptx::mapa(rml, (uint32_t)owner) + (uint32_t)((rank * rpc + rl) * 8);
+        asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(mdst), "f"(mml[r * 2]), "f"(mml[r * 2 + 1])
+                     : "memory");
+      }
+    }
+  }
+  if (trace && tid == 0) trace[6] = ptx::globaltimer();
   ptx::cluster_sync();
+  if (trace && tid == 0) trace[7] = ptx::globaltimer();
   // combine the ranks' partials for my rows, in rank order
   const int r0 = rank * rpc, n_own = min(a.S, r0 + rpc) - r0;
   if (tid < n_own) {
@@ -623,13 +702,15 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const AttnArgs a) {
     const int rl = idx / (D / 2), d2 = idx - rl * (D / 2);
     float ox = 0.f, oy = 0.f;
     for (int qr = 0; qr < nchunk; ++qr) {
-      const float2 v = *reinterpret_cast<const float2*>(recv + (qr * rpc + rl) * D + 2 * d2);
+      const float2 v = __bfloat1622float2(
+          *reinterpret_cast<const __nv_bfloat162*>(recv + (size_t)(qr * rpc + rl) * D + 2 * d2));
       ox = fmaf(wq_s[rl * nchunk + qr], v.x, ox);
       oy = fmaf(wq_s[rl * nchunk + qr], v.y, oy);
     }
     *reinterpret_cast<uint32_t*>(a.o + (((size_t)g * a.S + r0 + rl) * a.Hq + j) * D + 2 * d2) =
         ptx::pack_bf16x2(ox * inv_s[rl], oy * inv_s[rl]);
   }
+  if (trace && tid == 0) trace[8] = ptx::globaltimer();
 }
 
 // ---------------------------------------------------------------------------
@@ -807,10 +888,11 @@ struct FastPath {
   float* ssp = nullptr;
   int num_sms = 148;
   int max_cluster = 8;
+  int attn_fit[17] = {0};      // co-resident clusters of attention CTAs, by cluster size
   int smem_cap = 112 * 1024;   // keeps two CTAs per SM so the next kernel can prefetch
   // optional phase trace of the four projections of layer 0 in the first Euler step
   unsigned long long* trace = nullptr;
-  int trace_ctas[4] = {0, 0, 0, 0};
+  int trace_ctas[5] = {0, 0, 0, 0, 0};
   bool trace_armed = false;
   std::vector<void*> allocs;
 };
@@ -863,10 +945,12 @@ GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T) {
   }
   const int nbox = best.kslice / 64;
   int stages = nbox;
-  while (stages > 1 && gemm_smem_layout(stages, n_mma, best.cs, T).total > fp->smem_cap) --stages;
+  // a grid of at most one CTA per SM may use the whole shared memory for its ring
+  const int cap = best.n_tiles * best.cs <= fp->num_sms ? kDynSmemMax : fp->smem_cap;
+  while (stages > 1 && gemm_smem_layout(stages, n_mma, best.cs, T).total > cap) --stages;
   best.stages = stages;
   best.smem = gemm_smem_layout(stages, n_mma, best.cs, T).total;
-  best.valid = best.kslice >= 64 && best.smem <= kDynSmemMax;
+  best.valid = best.kslice >= 64 && best.smem <= kDynSmemMax && (T + best.cs - 1) / best.cs <= 64;
   return best;
 }
 
@@ -915,7 +999,29 @@ cudaError_t configure_gemm() {
 
 template <int D>
 cudaError_t configure_attn() {
-  return configure_dyn_smem(attn_mma_kernel<D>);
+  cudaError_t e = configure_dyn_smem(attn_mma_kernel<D>);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(attn_mma_kernel<D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
+}
+
+// How many clusters of `cs` attention CTAs can run at once on this device.
+template <int D>
+int attn_clusters_that_fit(int cs, int S) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = attn_smem_bytes(D, cs, (S + cs - 1) / cs);
+  cudaLaunchAttribute at;
+  at.id = cudaLaunchAttributeClusterDimension;
+  at.val.clusterDim.x = cs;
+  at.val.clusterDim.y = 1;
+  at.val.clusterDim.z = 1;
+  cfg.attrs = &at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, attn_mma_kernel<D>, &cfg) != cudaSuccess) n = 0;
+  cudaGetLastError();
+  return n;
 }
 
 template <int D>
@@ -952,8 +1058,17 @@ cudaError_t launch_step(const StepArgs& a, int rows, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, step_kernel, a);
 }
 
-// Attention split: the cluster's ranks take ~equal key ranges (tiles of 128 keys).
-int attn_chunks(int nk) { return std::max(1, std::min(8, (nk + 63) / 64)); }
+// Attention split: the largest cluster (at most one rank per 32 keys) of
+// which every (head, suffix) pair's cluster can run at once; ranks take
+// ~equal key ranges.
+int attn_chunks(const FastPath* fp, int nk, int n_clusters) {
+  const int cap = std::max(1, (nk + 31) / 32);
+  for (int c : {16, 12, 8, 6, 4, 2}) {
+    if (c > cap) continue;
+    if (fp->attn_fit[c] >= n_clusters) return c;
+  }
+  return std::max(1, std::min(8, cap));
+}
 
 }  // namespace
 
@@ -993,6 +1108,8 @@ rtv_status fast_create(rtv_ctx* ctx) {
     if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n >= 8) fp->max_cluster = 16;
     cudaGetLastError();
   }
+  for (int c : {2, 4, 6, 8, 12, 16})
+    fp->attn_fit[c] = k.head_dim == 256 ? attn_clusters_that_fit<256>(c, S) : attn_clusters_that_fit<128>(c, S);
   const size_t T = ctx->Tmax;
   auto alloc = [&](void** p, size_t bytes) -> bool {
     if (cudaMalloc(p, bytes) != cudaSuccess) return false;
@@ -1010,9 +1127,9 @@ rtv_status fast_create(rtv_ctx* ctx) {
     return RTV_ERR_OOM;
   }
   if (getenv("RTV_TRACE")) {
-    if (cudaMalloc(&fp->trace, 4 * 512 * 16 * sizeof(unsigned long long)) == cudaSuccess) {
+    if (cudaMalloc(&fp->trace, 5 * 512 * 16 * sizeof(unsigned long long)) == cudaSuccess) {
       fp->allocs.push_back(fp->trace);
-      cudaMemset(fp->trace, 0, 4 * 512 * 16 * sizeof(unsigned long long));
+      cudaMemset(fp->trace, 0, 5 * 512 * 16 * sizeof(unsigned long long));
     } else {
       fp->trace = nullptr;
     }
@@ -1030,18 +1147,27 @@ void fast_arm_trace(rtv_ctx* ctx) {
 void fast_trace_report(rtv_ctx* ctx) {
   FastPath* fp = ctx->fast;
   if (!fp || !fp->trace || !fp->trace_ctas[0]) return;
-  std::vector<unsigned long long> h(4 * 512 * 16);
+  std::vector<unsigned long long> h(5 * 512 * 16);
   cudaDeviceSynchronize();
   cudaMemcpy(h.data(), fp->trace, h.size() * 8, cudaMemcpyDeviceToHost);
-  const char* nm[4] = {"qkv", "o", "gu", "down"};
-  const char* ev[9] = {"start", "w_issued", "pdl", "first_full", "mma_issued", "done", "copied", "recv", "end"};
+  const char* nm[5] = {"qkv", "o", "gu", "down", "attention"};
+  const char* ev[2][13] = {{"start", "w_issued", "pdl", "first_full", "mma_issued", "done", "copied", "recv", "end",
+                           "prefetched", "arrived", "iter0", "exit"},
+                          {"start", "pdl", "tile0", "loop_end", "merged", "entry", "pushed", "synced", "end", "", "", "",
+                           ""}};
   unsigned long long t_ref = ~0ull;
-  for (int i = 0; i < 4; ++i)
-    for (int c = 0; c < fp->trace_ctas[i]; ++c) t_ref = std::min(t_ref, h[((size_t)i * 512 + c) * 16]);
-  for (int i = 0; i < 4; ++i) {
-    fprintf(stderr, "[rtv trace] %s (%d CTAs), us after the first QKV CTA start: min / median / max\n", nm[i],
+  for (int i = 0; i < 5; ++i)
+    for (int c = 0; c < fp->trace_ctas[i]; ++c)
+      if (h[((size_t)i * 512 + c) * 16]) t_ref = std::min(t_ref, h[((size_t)i * 512 + c) * 16]);
+  const int order[5] = {0, 4, 1, 2, 3};
+  for (int oi = 0; oi < 5; ++oi) {
+    const int i = order[oi];
+    fprintf(stderr, "[rtv trace] %s (%d CTAs), us after the first traced start: min / median / max\n", nm[i],
             fp->trace_ctas[i]);
-    for (int e = 0; e < 9; ++e) {
+    const int order_e[13] = {0, 1, 2, 3, 4, 5, 6, 9, 7, 10, 11, 8, 12};
+    for (int ei = 0; ei < 13; ++ei) {
+      const int e = order_e[ei];
+      if (!ev[i == 4][e][0]) continue;
       std::vector<double> v;
       for (int c = 0; c < fp->trace_ctas[i]; ++c) {
         const unsigned long long t = h[((size_t)i * 512 + c) * 16 + e];
@@ -1049,15 +1175,12 @@ void fast_trace_report(rtv_ctx* ctx) {
       }
       if (v.empty()) continue;
       std::sort(v.begin(), v.end());
-      fprintf(stderr, "    %-11s %8.2f %8.2f %8.2f\n", ev[e], v.front(), v[v.size() / 2], v.back());
+      fprintf(stderr, "    %-11s %8.2f %8.2f %8.2f\n", ev[i == 4][e], v.front(), v[v.size() / 2], v.back());
     }
   }
 }
 
-bool fast_supports_prefix(rtv_ctx* ctx, int prefix_len) {
-  const int nk = prefix_len + ctx->S;
-  return (nk + attn_chunks(nk) - 1) / attn_chunks(nk) <= 8 * 128;
-}
+bool fast_supports_prefix(rtv_ctx*, int) { return true; }
 
 rtv_status fast_load(rtv_ctx* ctx, const rtv_tensor*, int) {
   FastPath* fp = ctx->fast;
@@ -1162,7 +1285,7 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
   const GemmPlan p_gu = plan_gemm(fp, 2 * F, w, n_mma, T);
   const GemmPlan p_dn = plan_gemm(fp, w, F, n_mma, T);
   const int nk = P + S;
-  const int nchunk = attn_chunks(nk);
+  const int nchunk = attn_chunks(fp, nk, k.n_q_heads * G);
   if (!(p_qkv.valid && p_o.valid && p_gu.valid && p_dn.valid) ||
       attn_smem_bytes(D, nchunk, (S + nchunk - 1) / nchunk) > kDynSmemMax) {
     ctx->last_error = "no tensor-core split fits this token count";
@@ -1181,9 +1304,9 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     for (int i = 0; i < 4; ++i)
       fprintf(stderr, "[rtv] T=%d %s: tiles=%d cluster=%d kslice=%d stages=%d smem=%d\n", T, nm[i], pls[i]->n_tiles,
               pls[i]->cs, pls[i]->kslice, pls[i]->stages, pls[i]->smem);
-    fprintf(stderr, "[rtv] attention: chunks=%d keys/chunk=%d smem=%d max_cluster=%d sms=%d\n", nchunk,
-            (nk + nchunk - 1) / nchunk, attn_smem_bytes(D, nchunk, (S + nchunk - 1) / nchunk), fp->max_cluster,
-            fp->num_sms);
+    fprintf(stderr, "[rtv] attention: chunks=%d keys/chunk=%d smem=%d max_cluster=%d sms=%d fit(8,12,16)=%d,%d,%d\n",
+            nchunk, (nk + nchunk - 1) / nchunk, attn_smem_bytes(D, nchunk, (S + nchunk - 1) / nchunk), fp->max_cluster,
+            fp->num_sms, fp->attn_fit[8], fp->attn_fit[12], fp->attn_fit[16]);
   }
 
   GemmArgs base{};
@@ -1232,6 +1355,7 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     fp->trace_ctas[1] = p_o.n_tiles * p_o.cs;
     fp->trace_ctas[2] = p_gu.n_tiles * p_gu.cs;
     fp->trace_ctas[3] = p_dn.n_tiles * p_dn.cs;
+    fp->trace_ctas[4] = nchunk * k.n_q_heads * G;
   }
   auto tr = [&](int l, int i) -> unsigned long long* {
     return (tracing && l == 0) ? fp->trace + (size_t)i * 512 * 16 : nullptr;
@@ -1244,6 +1368,7 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     a.w_row0 = l * nq;
     cudaError_t e = launch_gemm<GM_QKV>(fp->map_qkv, m_h, a, p_qkv, st);
 
+    at.trace = tr(l, 4);
     at.pk = (const __nv_bfloat16*)ctx->prefix_kv + (size_t)(2 * l) * kv_layer;
     at.pv = (const __nv_bfloat16*)ctx->prefix_kv + (size_t)(2 * l + 1) * kv_layer;
     if (e == cudaSuccess) e = D == 256 ? launch_attn<256>(at, nchunk, G, st) : launch_attn<128>(at, nchunk, G, st);
