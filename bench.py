@@ -50,6 +50,8 @@ def parse_args(argv=None):
     ap.add_argument("--n-steps", type=int, default=10, help="Euler steps per chunk")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds of the oracle sample")
+    ap.add_argument("--trace", action="store_true",
+                    help="print the library's phase stamps of layer 0 of the first Euler step (no timing)")
     return ap.parse_args(argv)
 
 
@@ -338,8 +340,27 @@ def run_ours(args, info):
     print(json.dumps(line), flush=True)
 
 
+def run_trace(args):
+    """One traced chunk: the library prints per-CTA phase stamps (globaltimer)
+    of the projections and the attention of layer 0, first Euler step."""
+    os.environ["RTV_TRACE"] = "1"
+    from flow_matching_action_dm0_b200 import ActionExpert
+    from synthetic import get_config, make_noise, make_prefix_kv, make_state, make_weights
+    cfg = get_config(args.workload, n_steps=args.n_steps)
+    ex = ActionExpert(cfg, max_batch=cfg.batch, max_taus=4)
+    ex.load(make_weights(cfg))
+    ex.set_prefix_kv(make_prefix_kv(cfg))
+    noise, state = make_noise(cfg), make_state(cfg)
+    for _ in range(max(3, args.warmup)):
+        ex.denoise(noise, state, cfg.n_steps)
+    ex.close()
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.trace:
+        run_trace(args)
+        return 0
     from flow_matching_action_dm0_b200 import replicas as R
     info = R.rank_info()
     if args.impl == "reference":

@@ -24,6 +24,12 @@ and section:
            the full path).
   [RTVLA]  "Running VLAs at Real-time Speed": 10 iterations of tens of layers.
 
+Pins: every elementary function is pinned in tests/test_oracle_pins.py
+against closed forms, brute force or library routines.  expert_velocity
+(the composed random-weight expert): parity unpinned by the pages, which
+print no worked numerical example; it is pinned only through its parts, the
+zero-layer closed form and an independent PyTorch restatement.
+
 Where the pages are silent the plainest reading is taken:
   R1 Euler sign: x <- x - dt*v with dt = 1/N, t_k = 1 - k/N (integrating from
      noise at t=1 to data at t=0 under u = eps - a).
