@@ -25,7 +25,8 @@ RTV_FLAG_ZERO_ACCEPT, RTV_FLAG_SWITCH, RTV_FLAG_SWITCH_IN_PREFIX = 1, 2, 4
 
 # Every symbol include/rtv.h declares (checked by the CPU test suite).
 EXPORTS = ("rtv_create", "rtv_load_expert", "rtv_set_prefix_kv", "rtv_denoise", "rtv_verify",
-           "rtv_device_status", "rtv_last_error", "rtv_path_name", "rtv_graph_kernel_count", "rtv_destroy")
+           "rtv_device_status", "rtv_last_error", "rtv_path_name", "rtv_graph_kernel_count", "rtv_destroy",
+           "rtv_set_prefix_kv_static")
 
 
 class rtv_expert_config(C.Structure):
@@ -66,6 +67,7 @@ def load_library(path: str = LIB_PATH):
     lib.rtv_create.argtypes = [C.POINTER(rtv_expert_config), I, C.POINTER(P)]
     lib.rtv_load_expert.argtypes = [P, C.POINTER(rtv_tensor), I]
     lib.rtv_set_prefix_kv.argtypes = [P, P, I, I, P]
+    lib.rtv_set_prefix_kv_static.argtypes = [P, P, I, I, P]
     lib.rtv_denoise.argtypes = [P, P, P, I, P, P]
     lib.rtv_verify.argtypes = [P, P, P, P, P, I, F, I, P, P, P, P]
     lib.rtv_device_status.argtypes = [P, U]
@@ -77,8 +79,8 @@ def load_library(path: str = LIB_PATH):
     lib.rtv_graph_kernel_count.restype = I
     lib.rtv_destroy.argtypes = [P]
     lib.rtv_destroy.restype = None
-    for n in ("rtv_create", "rtv_load_expert", "rtv_set_prefix_kv", "rtv_denoise", "rtv_verify",
-              "rtv_device_status"):
+    for n in ("rtv_create", "rtv_load_expert", "rtv_set_prefix_kv", "rtv_set_prefix_kv_static", "rtv_denoise",
+              "rtv_verify", "rtv_device_status"):
         getattr(lib, n).restype = I
     _lib = lib
     return lib
@@ -108,6 +110,12 @@ def rtv_load_expert(h, tensors):
 
 def rtv_set_prefix_kv(h, kv_ptr: int, prefix_len: int, batch: int, stream: int = 0):
     return _check(h, load_library().rtv_set_prefix_kv(h, C.c_void_p(kv_ptr), prefix_len, batch, C.c_void_p(stream)))
+
+
+def rtv_set_prefix_kv_static(h, kv_ptr: int, prefix_len: int, batch: int, stream: int = 0):
+    """Like rtv_set_prefix_kv, staging host data through the library's static device array (no allocation)."""
+    return _check(h, load_library().rtv_set_prefix_kv_static(h, C.c_void_p(kv_ptr), prefix_len, batch,
+                                                             C.c_void_p(stream)))
 
 
 def rtv_denoise(h, noise_ptr: int, state_ptr: int, n_steps: int, out_ptr: int, stream: int = 0):

@@ -145,6 +145,23 @@ rtv_status rtv_load_expert(rtv_ctx* ctx, const rtv_tensor* params, int n_params)
  * of [DM0.5] 6.5).  prefix_len <= max_prefix_len, batch <= max_batch. */
 rtv_status rtv_set_prefix_kv(rtv_ctx* ctx, const void* kv, int prefix_len, int batch, rtv_stream stream);
 
+/* Install the prefix KV cache without allocating any device memory.  No
+ * counterpart in the pages: this is a service for callers that cannot call
+ * cudaMalloc while running (a real-time control loop that must not block on
+ * the allocator, or a process whose device memory belongs to another
+ * allocator or a fixed budget).  Same arguments and result as
+ * rtv_set_prefix_kv; a host-resident `kv` is staged one layer at a time
+ * through a fixed 4 MiB array in device global memory that the library
+ * declares statically (every GPU that loads the library holds it until the
+ * process exits).  Returns RTV_ERR_SHAPE when one layer's keys and values
+ * (2 * batch * prefix_len * n_kv_heads * head_dim elements) exceed 4 MiB.
+ * The first call on a device looks up the array's device address; make that
+ * first call before any stream capture.  All calls share the array and it
+ * keeps the last call's contents: calls whose work overlaps on the GPU (other
+ * streams or other contexts on the same device) race on it, so serialise
+ * them.  Calls no cudaMalloc, cudaFree or allocating library routine. */
+rtv_status rtv_set_prefix_kv_static(rtv_ctx* ctx, const void* kv, int prefix_len, int batch, rtv_stream stream);
+
 /* Denoise ([DM0.5] 5.3): from noise x_1 = noise [batch][H][A], run n_steps
  * Euler steps x <- x - (1/n_steps) * v(x, t_k), t_k = 1 - k/n_steps, and
  * write the action chunk [batch][H][A] to actions_out.  state is
