@@ -18,10 +18,12 @@
 // out[t][n] = sum_k act[t][k] W[n][k], computed swapped, D = W x act^T, so
 // that 128 weight rows fill the tcgen05 M dimension and the tokens (padded to
 // a multiple of 16) form N.  A CTA owns one 128-row weight tile and one K
-// slice.  Its first ring-full of weight boxes is fetched by TMA as soon as the
-// CTA starts -- before it waits on the previous kernel, since weights do not
+// slice.  Its first ring-full of weight boxes is fetched as soon as the CTA
+// starts -- before it waits on the previous kernel, since weights do not
 // depend on it -- and the bf16 activation boxes follow once that kernel has
-// finished.  The K slices of one weight tile form a thread-block cluster: each
+// finished.  Weights and activations are stored tiled and pre-swizzled (see
+// ts_offset), so every box is one contiguous bulk copy that lands in shared
+// memory as a ready tensor-core operand.  The K slices of one weight tile form a thread-block cluster: each
 // rank copies the partial sums of the tokens another rank owns into that
 // rank's shared memory with one bulk copy, and the owner reduces them in rank
 // order (deterministic).
@@ -53,9 +55,23 @@ namespace rtv {
 
 enum { GM_QKV = 0, GM_O = 1, GM_GU = 2, GM_DOWN = 3 };
 
+// Element offset of (row t, column k) of a bf16 operand [rows][K] stored
+// tiled and pre-swizzled: blocks of `block_rows` rows x 64 columns (128-byte
+// rows, stacked densely), and inside a block the eight 16-byte chunks of row
+// t permuted as chunk ^ (t % 8) -- the order in which the tensor cores' 128-byte
+// swizzle reads a K-major operand.  A block copied byte for byte to a
+// 1024-byte-aligned shared-memory address is therefore a ready operand tile.
+// Activations use one block column per 64 inputs ([K/64][n_mma][64]);
+// weights use 128-row tiles ([R/128][K/64][128][64]).
+__host__ __device__ __forceinline__ size_t ts_offset(int t, int k, int block_rows) {
+  return ((size_t)(k >> 6) * block_rows + t) * 64 + ((((k >> 3) & 7) ^ (t & 7)) << 3) + (k & 7);
+}
+
 struct GemmArgs {
+  const __nv_bfloat16* wt;    // packed weights of this projection, all layers [R/128][K/64][128][64]
+  const __nv_bfloat16* act;   // bf16 input, tiled [K/64][n_mma][64]
   float* h;                   // fp32 residual stream [T][w] (O, DOWN add into it)
-  __nv_bfloat16* hb;          // next norm's input bf16(h * (1 + g_next)) [T][w]   (written by O, DOWN)
+  __nv_bfloat16* hb;          // next norm's input bf16(h * (1 + g_next)), tiled [w/64][n_mma][64] (written by O, DOWN)
   float* ssp;                 // sums of squares of h per 128-feature tile [T][w/128]
   const float* g_next;        // gain of the next RMSNorm, or nullptr when no norm consumer follows
   __nv_bfloat16* q;           // [T][Hq][D]
@@ -63,17 +79,19 @@ struct GemmArgs {
   __nv_bfloat16* vs;          // suffix values [G][Hkv][S][D]
   const float* rope_cs;       // [S][D/2]
   const float* rope_sn;
-  __nv_bfloat16* m;           // [T][F]
+  __nv_bfloat16* m;           // gelu(gate) * up, tiled [F/64][n_mma][64]
   unsigned* status;
   unsigned long long* trace;  // optional phase stamps [cta][16] (globaltimer ns), or nullptr
   long long timeout_ns;
-  int T, n_mma, kslice, stages, w, S, Hq, Hkv, D, F, w_row0;
+  int T, n_mma, kslice, stages, w, S, Hq, Hkv, D, F, K, w_tile0;
   float eps;
 };
 
-// Phase stamps of the optional trace (one row of 16 per CTA).
+// Phase stamps of the optional trace (one row of kTraceRow per CTA; GEMM
+// rows also hold the landing time of the first 8 stages from slot 16 on).
+constexpr int kTraceRow = 32;
 enum { TR_START = 0, TR_W_ISSUED, TR_PDL, TR_FIRST_FULL, TR_MMA_ISSUED, TR_DONE, TR_COPIED, TR_RECV, TR_END,
-       TR_PREFETCHED, TR_ARRIVED, TR_ITER0, TR_EXIT };
+       TR_PREFETCHED, TR_ARRIVED, TR_ITER0, TR_EXIT, TR_PART, TR_ENTRY };
 
 struct GemmSmem {
   int stages, stage_bytes, ring_bytes, part_off, recv_off, in_off, bar_off, total;
@@ -119,9 +137,6 @@ __device__ __forceinline__ uint32_t dynamic_smem_size() {
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void cluster_arrive_release() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 
 // Bulk copy of `bytes` from this CTA's shared memory to another CTA's shared
@@ -136,8 +151,7 @@ __device__ __forceinline__ void bulk_copy_to_rank(uint32_t dst_cluster, uint32_t
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap wmap,
-                                                         const __grid_constant__ CUtensorMap amap, const GemmArgs a) {
+__global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ float rs_s[64];
   const int n_mma = a.n_mma;
@@ -168,7 +182,10 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
   uint32_t* tmem_slot = (uint32_t*)(rbar + 1);
   const uint32_t ncols = (uint32_t)tmem_cols_for(n_mma);
   const uint32_t act_box_bytes = (uint32_t)n_mma * 128u;
-  unsigned long long* trace = a.trace ? a.trace + ((size_t)blockIdx.y * gridDim.x + blockIdx.x) * 16 : nullptr;
+  // this CTA's first weight box and first activation box
+  const __nv_bfloat16* wsrc = a.wt + ((size_t)(a.w_tile0 + nt) * (a.K >> 6) + (k0 >> 6)) * 8192;
+  const __nv_bfloat16* asrc = a.act + (size_t)(k0 >> 6) * n_mma * 64;
+  unsigned long long* trace = a.trace ? a.trace + ((size_t)blockIdx.y * gridDim.x + blockIdx.x) * kTraceRow : nullptr;
   if (trace && threadIdx.x == 0) trace[TR_START] = ptx::globaltimer();
 
   if (threadIdx.x == 0) {
@@ -194,7 +211,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       pol = ptx::policy_evict_first();
       for (int b = 0; b < first; ++b) {
         ptx::mbar_expect_tx(&full[b], 16384u);
-        ptx::tma_load_2d(base + b * L.stage_bytes, &wmap, &full[b], k0 + 64 * b, a.w_row0 + nt * 128, pol);
+        ptx::bulk_load_hint(base + b * L.stage_bytes, wsrc + (size_t)b * 8192, 16384u, &full[b], pol);
       }
       if (trace) trace[TR_W_ISSUED] = ptx::globaltimer();
     }
@@ -224,10 +241,10 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
             break;
           }
           ptx::mbar_expect_tx(&full[s], 16384u);
-          ptx::tma_load_2d(st, &wmap, &full[s], k0 + 64 * b, a.w_row0 + nt * 128, pol);
+          ptx::bulk_load_hint(st, wsrc + (size_t)b * 8192, 16384u, &full[s], pol);
         }
         ptx::mbar_expect_tx(&full[s], act_box_bytes);
-        ptx::tma_load_2d_nohint(st + 16384, &amap, &full[s], k0 + 64 * b, 0);
+        ptx::bulk_load(st + 16384, asrc + (size_t)b * n_mma * 64, act_box_bytes, &full[s]);
       }
     }
   } else if (warp == 1) {
@@ -242,6 +259,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
         }
         ptx::tc_fence_after();
         if (trace && b == 0) trace[TR_FIRST_FULL] = ptx::globaltimer();
+        if (trace && b < 8) trace[16 + b] = ptx::globaltimer();
         const uint32_t wa = ptx::smem_u32(base + s * L.stage_bytes);
         const uint32_t aa = wa + 16384u;
 #pragma unroll
@@ -260,40 +278,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     const int tid = threadIdx.x - 64;
     ptx::pdl_wait();   // this role reads and writes what earlier kernels produced
     if (tid == 0) ptx::mbar_expect_tx(rbar, (uint32_t)(cs * n_own * 512));
-    if (!ptx::mbar_wait(done, 0, a.timeout_ns)) atomicOr(a.status, RTV_DEV_TIMEOUT);
-    ptx::tc_fence_after();
-    if (trace && tid == 0) trace[TR_DONE] = ptx::globaltimer();
-    // accumulator -> this CTA's partial tile [token][feature]
-    const int quarter = warp & 3;
-    const int f = quarter * 32 + lane;
-    for (int c = 0; c < n_mma; c += 32) {
-      float v[32];
-      if (c + 16 < n_mma) {
-        ptx::tmem_ld_32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) part[(c + i) * 128 + f] = v[i];
-      } else {
-        ptx::tmem_ld_16(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c, *reinterpret_cast<float(*)[16]>(v));
-#pragma unroll
-        for (int i = 0; i < 16; ++i) part[(c + i) * 128 + f] = v[i];
-      }
-    }
-    ptx::tc_fence_before();
-    ptx::fence_proxy_async_smem();
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    cluster_wait();   // entry phase: every rank has started and initialised its barriers
-    if (tid == 0) {
-      const uint32_t part_a = ptx::smem_u32(part), recv_a = ptx::smem_u32(recv), rbar_a = ptx::smem_u32(rbar);
-      for (int r = 0; r < cs; ++r) {
-        const int o0 = r * per, no = max(0, min(a.T, o0 + per) - o0);
-        if (no == 0) continue;
-        bulk_copy_to_rank(ptx::mapa(recv_a + (uint32_t)(rank * per * 512), (uint32_t)r),
-                          part_a + (uint32_t)(o0 * 512), (uint32_t)(no * 512), ptx::mapa(rbar_a, (uint32_t)r));
-      }
-      if (trace) trace[TR_COPIED] = ptx::globaltimer();
-    }
-    // Everything the epilogue reads from global memory is requested now, in
-    // parallel, while the partials are still in flight: the owned tokens'
+    // Everything the epilogue reads from global memory depends only on earlier
+    // kernels, so it is requested now, while the MMAs run: the owned tokens'
     // residual rows of this tile (O, DOWN) or their RoPE cos/sin (QKV) go to
     // shared memory by cp.async; 1/rms of the owned tokens (QKV, GU) too.
     float* in_s = (float*)(base + L.in_off);
@@ -315,22 +301,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
         ptx::cp_async_16(in_a + (uint32_t)(c * 16), src);
       }
     }
-    if ((MODE == GM_QKV || MODE == GM_GU) && tid < n_own) {
-      float sst = 0.f;
-      for (int j2 = 0; j2 < n_wt; ++j2) sst += a.ssp[(size_t)(t_own0 + tid) * n_wt + j2];
-      rs_s[tid] = rsqrtf(sst / (float)a.w + a.eps);
-    }
-    ptx::cp_async_wait_all();
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (trace && tid == 0) trace[TR_PREFETCHED] = ptx::globaltimer();
-    if (!ptx::mbar_wait(rbar, 0, a.timeout_ns)) atomicOr(a.status, RTV_DEV_TIMEOUT);
-    if (trace && tid == 0) trace[TR_RECV] = ptx::globaltimer();
-    cluster_arrive_release();   // my incoming copies are complete
-    if (trace && tid == 0) trace[TR_ARRIVED] = ptx::globaltimer();
-
-    // ---- reduction in rank order + epilogue for the tokens this rank owns ----
-    // one warp per token; lane l takes features (2l, 2l+1) and (2l+64, 2l+65)
-    const int ew = warp - 2;
+    // gains of the next norm for this lane's features (O, DOWN)
     const int f0 = 2 * lane;
     const int n1 = nt * 128 + f0, n2 = n1 + 64;
     float2 gn1 = make_float2(0.f, 0.f), gn2 = make_float2(0.f, 0.f);
@@ -338,6 +309,58 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       gn1 = *reinterpret_cast<const float2*>(a.g_next + n1);
       gn2 = *reinterpret_cast<const float2*>(a.g_next + n2);
     }
+    if ((MODE == GM_QKV || MODE == GM_GU) && tid < n_own) {
+      float sst = 0.f;
+      for (int j2 = 0; j2 < n_wt; ++j2) sst += a.ssp[(size_t)(t_own0 + tid) * n_wt + j2];
+      rs_s[tid] = rsqrtf(sst / (float)a.w + a.eps);
+    }
+    if (!ptx::mbar_wait(done, 0, a.timeout_ns)) atomicOr(a.status, RTV_DEV_TIMEOUT);
+    ptx::tc_fence_after();
+    if (trace && tid == 0) trace[TR_DONE] = ptx::globaltimer();
+    // accumulator -> this CTA's partial tile [token][feature]
+    const int quarter = warp & 3;
+    const int f = quarter * 32 + lane;
+    for (int c = 0; c < n_mma; c += 32) {
+      float v[32];
+      if (c + 16 < n_mma) {
+        ptx::tmem_ld_32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) part[(c + i) * 128 + f] = v[i];
+      } else {
+        ptx::tmem_ld_16(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c, *reinterpret_cast<float(*)[16]>(v));
+#pragma unroll
+        for (int i = 0; i < 16; ++i) part[(c + i) * 128 + f] = v[i];
+      }
+    }
+    ptx::tc_fence_before();
+    ptx::fence_proxy_async_smem();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (trace && tid == 0) trace[TR_PART] = ptx::globaltimer();
+    cluster_wait();   // entry phase: every rank has started and initialised its barriers
+    if (trace && tid == 0) trace[TR_ENTRY] = ptx::globaltimer();
+    if (tid == 0) {
+      const uint32_t part_a = ptx::smem_u32(part), recv_a = ptx::smem_u32(recv), rbar_a = ptx::smem_u32(rbar);
+      for (int r = 0; r < cs; ++r) {
+        const int o0 = r * per, no = max(0, min(a.T, o0 + per) - o0);
+        if (no == 0) continue;
+        bulk_copy_to_rank(ptx::mapa(recv_a + (uint32_t)(rank * per * 512), (uint32_t)r),
+                          part_a + (uint32_t)(o0 * 512), (uint32_t)(no * 512), ptx::mapa(rbar_a, (uint32_t)r));
+      }
+      if (trace) trace[TR_COPIED] = ptx::globaltimer();
+    }
+    ptx::cp_async_wait_all();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (trace && tid == 0) trace[TR_PREFETCHED] = ptx::globaltimer();
+    if (!ptx::mbar_wait(rbar, 0, a.timeout_ns)) atomicOr(a.status, RTV_DEV_TIMEOUT);
+    if (trace && tid == 0) trace[TR_RECV] = ptx::globaltimer();
+    // My incoming copies are complete (seen on rbar), so the copies that read
+    // the senders' shared memory are done too; the arrive needs no ordering.
+    cluster_arrive_relaxed();
+    if (trace && tid == 0) trace[TR_ARRIVED] = ptx::globaltimer();
+
+    // ---- reduction in rank order + epilogue for the tokens this rank owns ----
+    // one warp per token; lane l takes features (2l, 2l+1) and (2l+64, 2l+65)
+    const int ew = warp - 2;
 #pragma unroll 1
     for (int tl = ew; tl < n_own; tl += 4) {
       const int t = t_own0 + tl;
@@ -365,9 +388,9 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
           sq = fmaf(h2.x, h2.x, sq);
           sq = fmaf(h2.y, h2.y, sq);
           sq = warp_sum(sq);
-          *reinterpret_cast<uint32_t*>(a.hb + (size_t)t * a.w + n1) =
+          *reinterpret_cast<uint32_t*>(a.hb + ts_offset(t, n1, n_mma)) =
               ptx::pack_bf16x2(h1.x * (1.f + gn1.x), h1.y * (1.f + gn1.y));
-          *reinterpret_cast<uint32_t*>(a.hb + (size_t)t * a.w + n2) =
+          *reinterpret_cast<uint32_t*>(a.hb + ts_offset(t, n2, n_mma)) =
               ptx::pack_bf16x2(h2.x * (1.f + gn2.x), h2.y * (1.f + gn2.y));
           if (lane == 0) a.ssp[(size_t)t * n_wt + nt] = sq;
         }
@@ -378,7 +401,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
         x2.x *= rs;
         x2.y *= rs;
         if (MODE == GM_GU) {
-          *reinterpret_cast<uint32_t*>(a.m + (size_t)t * a.F + nt * 64 + f0) =
+          *reinterpret_cast<uint32_t*>(a.m + ts_offset(t, nt * 64 + f0, n_mma)) =
               ptx::pack_bf16x2(gelu_tanh(x1.x) * x2.x, gelu_tanh(x1.y) * x2.y);
         } else {
           const int g = t / a.S, s = t - g * a.S;
@@ -403,7 +426,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
   }
   if (warp < 2) {
     cluster_wait();             // entry phase
-    cluster_arrive_release();   // nothing incoming to wait for
+    cluster_arrive_relaxed();   // nothing incoming to wait for
   }
   cluster_wait();   // every rank's incoming copies are complete: no copy still reads my shared memory
   if (trace && threadIdx.x == 64) trace[TR_EXIT] = ptx::globaltimer();
@@ -422,11 +445,12 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
 // ("DM0.5 reading guide", sec. 5.1-5.2: suffix queries over the cached prefix
 // KV and the bidirectional suffix; optional Pi0 block mask for the state
 // token).  The cluster's CTAs take consecutive key ranges of [prefix ; own
-// suffix] in tiles of 128 keys.  In a CTA, warp w handles query rows
-// 16*(w%4).. and one 64-key half of each tile with a flash-style online
-// softmax on warp-level bf16 MMAs (fp32 accumulate).  The two halves are
-// merged in shared memory, then every CTA pushes its (max, sum, partial
-// output) rows to the rank that combines them.
+// suffix] in tiles of 64 keys; warp w of a CTA owns query rows 16w..16w+15
+// and runs a flash-style online softmax over all of the CTA's keys on
+// warp-level bf16 MMAs (fp32 accumulate).  Each CTA then writes its
+// unnormalised partial rows and their (max, sum) to global memory (they stay
+// in L2), the cluster synchronises, and every rank combines the rows it owns,
+// in rank order.
 // ---------------------------------------------------------------------------
 struct AttnArgs {
   const __nv_bfloat16* q;    // [T][Hq][D]
@@ -434,38 +458,34 @@ struct AttnArgs {
   const __nv_bfloat16* pv;   // this layer's prefix values
   const __nv_bfloat16* sk;   // suffix keys   [G][Hkv][S][D]
   const __nv_bfloat16* sv;
-  __nv_bfloat16* o;          // [T][Hq*D]
+  __nv_bfloat16* o;          // attention output, tiled [Hq*D/64][n_mma][64]
+  __nv_bfloat16* part_o;     // partial rows [G][Hq][nchunk][64][D] (scratch)
+  float* part_ml;            // their (max, sum) [G][Hq][nchunk][64][2]
   unsigned* status;
-  unsigned long long* trace; // optional phase stamps [cta][16], or nullptr
-  int S, P, Pmax, Hq, Hkv, pbs, mask_mode, kpc;
+  unsigned long long* trace; // optional phase stamps [cta][kTraceRow], or nullptr
+  int S, P, Pmax, Hq, Hkv, pbs, mask_mode, kpc, n_mma;
   float scale_log2;
 };
 
-// Q tile, K and V tiles, receive buffers of the cluster combine (bf16 rows +
-// fp32 max/sum), combine weights.
-__host__ __device__ inline int attn_smem_bytes(int D, int nchunk, int rpc) {
-  return 64 * D * 2 + 2 * 128 * D * 2 + nchunk * rpc * D * 2 + nchunk * rpc * 2 * 4 + rpc * (nchunk + 1) * 4;
-}
+// Q, K and V tiles of 64 rows; once a warp is done with the keys, its rows
+// of the Q tile stage its partial rows on their way to global memory.
+__host__ __device__ inline int attn_smem_bytes(int D) { return 3 * 64 * D * 2; }
 
 template <int D>
-__global__ void __launch_bounds__(256) attn_mma_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
   extern __shared__ __align__(128) uint8_t sm_attn[];
-  constexpr int CPR = D / 8;   // 16-byte chunks per row
+  constexpr int CPR = D / 8;           // 16-byte chunks per row
   const int nchunk = gridDim.x;
   const int rpc = (a.S + nchunk - 1) / nchunk;   // query rows combined by each rank
-  if (dynamic_smem_size() < (uint32_t)attn_smem_bytes(D, nchunk, rpc) || a.S > 64 || nchunk > 16) {
+  // every CTA of the grid sees the same values, so a refusal is uniform
+  if (dynamic_smem_size() < (uint32_t)attn_smem_bytes(D) || a.S > 64 || nchunk > 32) {
     if (threadIdx.x == 0) atomicOr(a.status, RTV_DEV_BOUNDS);
     return;
   }
   __nv_bfloat16* Qs = reinterpret_cast<__nv_bfloat16*>(sm_attn);
   __nv_bfloat16* Ks = Qs + 64 * D;
-  __nv_bfloat16* Vs = Ks + 128 * D;
-  __nv_bfloat16* recv = Vs + 128 * D;                      // [nchunk][rpc][D] partial outputs pushed to me
-  float* recv_ml = reinterpret_cast<float*>(recv + nchunk * rpc * D);   // [nchunk][rpc][2] (running max, sum)
-  float* wq_s = recv_ml + nchunk * rpc * 2;                 // [rpc][nchunk] combine weights
-  float* inv_s = wq_s + rpc * nchunk;                       // [rpc] 1 / combined sum
+  __nv_bfloat16* Vs = Ks + 64 * D;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int rb = warp & 3, kh = warp >> 2;
   const int rank = (int)ptx::cluster_ctarank();
   const int j = blockIdx.y, g = blockIdx.z;
   const int kvh = (j * a.Hkv) / a.Hq;
@@ -479,32 +499,18 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const AttnArgs a) {
   const __nv_bfloat16* svh = a.sv + ((size_t)g * a.Hkv + kvh) * a.S * D;
 
   unsigned long long* trace =
-      a.trace ? a.trace + (((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * 16 : nullptr;
+      a.trace ? a.trace + (((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * kTraceRow
+              : nullptr;
   if (trace && tid == 0) trace[0] = ptx::globaltimer();
-  cluster_arrive_relaxed();
   ptx::pdl_launch_dependents();
-  ptx::pdl_wait();
-  if (trace && tid == 0) trace[1] = ptx::globaltimer();
 
   const uint32_t qs_a = ptx::smem_u32(Qs), ks_a = ptx::smem_u32(Ks), vs_a = ptx::smem_u32(Vs);
-  for (int c = tid; c < 64 * CPR; c += 256) {
-    const int r = c / CPR, ch = c - r * CPR;
-    const uint32_t off = (uint32_t)((r * D + ((ch ^ (r & 7)) << 3)) * 2);
-    if (r < a.S) ptx::cp_async_16(qs_a + off, a.q + (((size_t)g * a.S + r) * a.Hq + j) * D + ch * 8);
-    else *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(Qs) + off) = make_uint4(0, 0, 0, 0);
-  }
-
-  float o_acc[D / 8][4];
-#pragma unroll
-  for (int i = 0; i < D / 8; ++i) o_acc[i][0] = o_acc[i][1] = o_acc[i][2] = o_acc[i][3] = 0.f;
-  float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
-  const int row0 = 16 * rb + (lane >> 2);
-
-  for (int kt = kb; kt < ke; kt += 128) {
-    __syncthreads();
-    for (int c = tid; c < 128 * CPR; c += 256) {
+  // K/V rows [lo, hi) of the 64-key tile starting at kt (keys past ke read as zeros)
+  auto load_kv = [&](int kt, int lo, int hi) {
+    for (int c = tid; c < 64 * CPR; c += 128) {
       const int r = c / CPR, ch = c - r * CPR;
       const int n = kt + r;
+      if (n < lo || n >= hi) continue;
       const uint32_t off = (uint32_t)((r * D + ((ch ^ (r & 7)) << 3)) * 2);
       if (n < ke) {
         const __nv_bfloat16* ksrc = n < a.P ? pkh + (size_t)n * D : skh + (size_t)(n - a.P) * D;
@@ -516,89 +522,114 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const AttnArgs a) {
         *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(Vs) + off) = make_uint4(0, 0, 0, 0);
       }
     }
+  };
+  // The cached prefix does not depend on the previous kernel: the first
+  // tile's prefix rows are requested before waiting on it.
+  const int p_end = min(a.P, ke);
+  load_kv(kb, kb, p_end);
+  ptx::pdl_wait();
+  if (trace && tid == 0) trace[1] = ptx::globaltimer();
+
+  for (int c = tid; c < 64 * CPR; c += 128) {
+    const int r = c / CPR, ch = c - r * CPR;
+    const uint32_t off = (uint32_t)((r * D + ((ch ^ (r & 7)) << 3)) * 2);
+    if (r < a.S) ptx::cp_async_16(qs_a + off, a.q + (((size_t)g * a.S + r) * a.Hq + j) * D + ch * 8);
+    else *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(Qs) + off) = make_uint4(0, 0, 0, 0);
+  }
+
+  float o_acc[D / 8][4];
+#pragma unroll
+  for (int i = 0; i < D / 8; ++i) o_acc[i][0] = o_acc[i][1] = o_acc[i][2] = o_acc[i][3] = 0.f;
+  float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
+  const int row0 = 16 * warp + (lane >> 2);
+
+  for (int kt = kb; kt < ke; kt += 64) {
+    if (kt == kb) {
+      load_kv(kt, p_end, kt + 64);   // suffix rows and the zero tail of the first tile
+    } else {
+      __syncthreads();
+      load_kv(kt, kt, kt + 64);
+    }
     ptx::cp_async_wait_all();
     __syncthreads();
     if (trace && tid == 0 && kt == kb) trace[2] = ptx::globaltimer();
-    const int kbase = 64 * kh;   // this warp's half of the tile
-    if (kt + kbase < ke) {
-      // scores S = Q K^T for this warp's 16 rows x 64 keys
-      float s_acc[8][4];
+    // scores S = Q K^T for this warp's 16 rows x 64 keys
+    float s_acc[8][4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) s_acc[i][0] = s_acc[i][1] = s_acc[i][2] = s_acc[i][3] = 0.f;
+    for (int i = 0; i < 8; ++i) s_acc[i][0] = s_acc[i][1] = s_acc[i][2] = s_acc[i][3] = 0.f;
 #pragma unroll 4
-      for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t af[4];
-        {
-          const int r = 16 * rb + (lane & 15), ch = 2 * kk + (lane >> 4);
-          ptx::ldmatrix_x4(af, qs_a + (uint32_t)((r * D + ((ch ^ (r & 7)) << 3)) * 2));
-        }
-#pragma unroll
-        for (int np = 0; np < 4; ++np) {
-          uint32_t bf[4];
-          const int r = kbase + 16 * np + (lane & 7) + ((lane >> 4) << 3), ch = 2 * kk + ((lane >> 3) & 1);
-          ptx::ldmatrix_x4(bf, ks_a + (uint32_t)((r * D + ((ch ^ (r & 7)) << 3)) * 2));
-          ptx::mma_bf16_16816(s_acc[2 * np], af, bf[0], bf[1]);
-          ptx::mma_bf16_16816(s_acc[2 * np + 1], af, bf[2], bf[3]);
-        }
-      }
-      // mask, scale, online softmax (base-2 exponent)
-      float tmax[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int key = kt + kbase + 8 * nt + 2 * (lane & 3) + (e & 1);
-          const int r = row0 + ((e >> 1) << 3);
-          const bool ok = key < ke && !(a.mask_mode == RTV_MASK_PI0_BLOCK && r == 0 && key > a.P);
-          const float sv = ok ? s_acc[nt][e] * a.scale_log2 : -INFINITY;
-          s_acc[nt][e] = sv;
-          tmax[e >> 1] = fmaxf(tmax[e >> 1], sv);
-        }
-      }
-      float corr[2], mnew[2];
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        tmax[i] = fmaxf(tmax[i], __shfl_xor_sync(0xffffffffu, tmax[i], 1));
-        tmax[i] = fmaxf(tmax[i], __shfl_xor_sync(0xffffffffu, tmax[i], 2));
-        mnew[i] = fmaxf(m_r[i], tmax[i]);
-        corr[i] = (m_r[i] == -INFINITY) ? (mnew[i] == -INFINITY ? 1.f : 0.f) : exp2f(m_r[i] - mnew[i]);
-        m_r[i] = mnew[i];
-        l_r[i] *= corr[i];
+    for (int kk = 0; kk < D / 16; ++kk) {
+      uint32_t af[4];
+      {
+        const int r = 16 * warp + (lane & 15), ch = 2 * kk + (lane >> 4);
+        ptx::ldmatrix_x4(af, qs_a + (uint32_t)((r * D + ((ch ^ (r & 7)) << 3)) * 2));
       }
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float pv = (s_acc[nt][e] == -INFINITY) ? 0.f : exp2f(s_acc[nt][e] - mnew[e >> 1]);
-          s_acc[nt][e] = pv;
-          l_r[e >> 1] += pv;
-        }
+      for (int np = 0; np < 4; ++np) {
+        uint32_t bf[4];
+        const int r = 16 * np + (lane & 7) + ((lane >> 4) << 3), ch = 2 * kk + ((lane >> 3) & 1);
+        ptx::ldmatrix_x4(bf, ks_a + (uint32_t)((r * D + ((ch ^ (r & 7)) << 3)) * 2));
+        ptx::mma_bf16_16816(s_acc[2 * np], af, bf[0], bf[1]);
+        ptx::mma_bf16_16816(s_acc[2 * np + 1], af, bf[2], bf[3]);
       }
-      if (kt != kb) {
+    }
+    // mask, scale, online softmax (base-2 exponent)
+    float tmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-        for (int i = 0; i < D / 8; ++i) {
-          o_acc[i][0] *= corr[0];
-          o_acc[i][1] *= corr[0];
-          o_acc[i][2] *= corr[1];
-          o_acc[i][3] *= corr[1];
-        }
+    for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = kt + 8 * nt + 2 * (lane & 3) + (e & 1);
+        const int r = row0 + ((e >> 1) << 3);
+        const bool ok = key < ke && !(a.mask_mode == RTV_MASK_PI0_BLOCK && r == 0 && key > a.P);
+        const float sv = ok ? s_acc[nt][e] * a.scale_log2 : -INFINITY;
+        s_acc[nt][e] = sv;
+        tmax[e >> 1] = fmaxf(tmax[e >> 1], sv);
       }
-      // O += P V
+    }
+    float corr[2], mnew[2];
 #pragma unroll
-      for (int kb2 = 0; kb2 < 4; ++kb2) {
-        uint32_t pf[4];
-        pf[0] = ptx::pack_bf16x2(s_acc[2 * kb2][0], s_acc[2 * kb2][1]);
-        pf[1] = ptx::pack_bf16x2(s_acc[2 * kb2][2], s_acc[2 * kb2][3]);
-        pf[2] = ptx::pack_bf16x2(s_acc[2 * kb2 + 1][0], s_acc[2 * kb2 + 1][1]);
-        pf[3] = ptx::pack_bf16x2(s_acc[2 * kb2 + 1][2], s_acc[2 * kb2 + 1][3]);
+    for (int i = 0; i < 2; ++i) {
+      tmax[i] = fmaxf(tmax[i], __shfl_xor_sync(0xffffffffu, tmax[i], 1));
+      tmax[i] = fmaxf(tmax[i], __shfl_xor_sync(0xffffffffu, tmax[i], 2));
+      mnew[i] = fmaxf(m_r[i], tmax[i]);
+      corr[i] = (m_r[i] == -INFINITY) ? (mnew[i] == -INFINITY ? 1.f : 0.f) : exp2f(m_r[i] - mnew[i]);
+      m_r[i] = mnew[i];
+      l_r[i] *= corr[i];
+    }
 #pragma unroll
-        for (int dn = 0; dn < D / 16; ++dn) {
-          uint32_t bf[4];
-          const int r = kbase + 16 * kb2 + (lane & 7) + (((lane >> 3) & 1) << 3), ch = 2 * dn + (lane >> 4);
-          ptx::ldmatrix_x4_trans(bf, vs_a + (uint32_t)((r * D + ((ch ^ (r & 7)) << 3)) * 2));
-          ptx::mma_bf16_16816(o_acc[2 * dn], pf, bf[0], bf[1]);
-          ptx::mma_bf16_16816(o_acc[2 * dn + 1], pf, bf[2], bf[3]);
-        }
+    for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float pv = (s_acc[nt][e] == -INFINITY) ? 0.f : exp2f(s_acc[nt][e] - mnew[e >> 1]);
+        s_acc[nt][e] = pv;
+        l_r[e >> 1] += pv;
+      }
+    }
+    if (kt != kb) {
+#pragma unroll
+      for (int i = 0; i < D / 8; ++i) {
+        o_acc[i][0] *= corr[0];
+        o_acc[i][1] *= corr[0];
+        o_acc[i][2] *= corr[1];
+        o_acc[i][3] *= corr[1];
+      }
+    }
+    // O += P V
+#pragma unroll
+    for (int kb2 = 0; kb2 < 4; ++kb2) {
+      uint32_t pf[4];
+      pf[0] = ptx::pack_bf16x2(s_acc[2 * kb2][0], s_acc[2 * kb2][1]);
+      pf[1] = ptx::pack_bf16x2(s_acc[2 * kb2][2], s_acc[2 * kb2][3]);
+      pf[2] = ptx::pack_bf16x2(s_acc[2 * kb2 + 1][0], s_acc[2 * kb2 + 1][1]);
+      pf[3] = ptx::pack_bf16x2(s_acc[2 * kb2 + 1][2], s_acc[2 * kb2 + 1][3]);
+#pragma unroll
+      for (int dn = 0; dn < D / 16; ++dn) {
+        uint32_t bf[4];
+        const int r = 16 * kb2 + (lane & 7) + (((lane >> 3) & 1) << 3), ch = 2 * dn + (lane >> 4);
+        ptx::ldmatrix_x4_trans(bf, vs_a + (uint32_t)((r * D + ((ch ^ (r & 7)) << 3)) * 2));
+        ptx::mma_bf16_16816(o_acc[2 * dn], pf, bf[0], bf[1]);
+        ptx::mma_bf16_16816(o_acc[2 * dn + 1], pf, bf[2], bf[3]);
       }
     }
   }
@@ -609,106 +640,71 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const AttnArgs a) {
     l_r[i] += __shfl_xor_sync(0xffffffffu, l_r[i], 1);
     l_r[i] += __shfl_xor_sync(0xffffffffu, l_r[i], 2);
   }
-  // merge the two key halves of each row block in shared memory (K/V tiles are dead)
-  __syncthreads();
-  // padded row strides keep the fragment-order accesses below free of bank conflicts
-  constexpr int XS = D + 8;                                      // fp32 row stride of xo
-  constexpr int OS = D + 8;                                      // bf16 row stride of ob_s
-  float* xo = reinterpret_cast<float*>(Ks);                      // [64 rows][XS] fp32   (K and V tiles are dead)
-  __nv_bfloat16* ob_s = reinterpret_cast<__nv_bfloat16*>(xo + 64 * XS);   // [64 rows][OS] merged rows, bf16
-  float* xml = reinterpret_cast<float*>(Qs);                     // [64 rows][2] (the Q tile is dead too)
-  float* mml = reinterpret_cast<float*>(Qs) + 64 * 2;            // [64 rows][2] merged (max, sum)
-  if (kh == 1) {
+  // This rank's partial rows: each warp stages its 16 rows (bf16,
+  // chunk-swizzled) in its own rows of the Q tile, which no other warp reads,
+  // then copies the valid ones to global memory with 16-byte stores.
+  __syncwarp();
 #pragma unroll
-    for (int nt = 0; nt < D / 8; ++nt) {
-      const int d = 8 * nt + 2 * (lane & 3);
-      *reinterpret_cast<float2*>(xo + row0 * XS + d) = make_float2(o_acc[nt][0], o_acc[nt][1]);
-      *reinterpret_cast<float2*>(xo + (row0 + 8) * XS + d) = make_float2(o_acc[nt][2], o_acc[nt][3]);
-    }
-    if ((lane & 3) == 0) {
-      xml[row0 * 2] = m_r[0];
-      xml[row0 * 2 + 1] = l_r[0];
-      xml[(row0 + 8) * 2] = m_r[1];
-      xml[(row0 + 8) * 2 + 1] = l_r[1];
-    }
-  }
-  __syncthreads();
-  if (kh == 0) {
+  for (int nt = 0; nt < D / 8; ++nt) {
 #pragma unroll
     for (int hrow = 0; hrow < 2; ++hrow) {
       const int r = row0 + 8 * hrow;
-      const float m2 = xml[r * 2], l2 = xml[r * 2 + 1];
-      const float mm = fmaxf(m_r[hrow], m2);
-      const float w1 = m_r[hrow] == -INFINITY ? 0.f : exp2f(m_r[hrow] - mm);
-      const float w2 = m2 == -INFINITY ? 0.f : exp2f(m2 - mm);
-#pragma unroll
-      for (int nt = 0; nt < D / 8; ++nt) {
-        const int d = 8 * nt + 2 * (lane & 3);
-        const float2 o2 = *reinterpret_cast<const float2*>(xo + r * XS + d);
-        *reinterpret_cast<uint32_t*>(ob_s + r * OS + d) =
-            ptx::pack_bf16x2(o_acc[nt][2 * hrow] * w1 + o2.x * w2, o_acc[nt][2 * hrow + 1] * w1 + o2.y * w2);
-      }
-      if ((lane & 3) == 0) {
-        mml[r * 2] = mm;
-        mml[r * 2 + 1] = l_r[hrow] * w1 + l2 * w2;
-      }
+      *reinterpret_cast<uint32_t*>(Qs + r * D + ((nt ^ (r & 7)) << 3) + 2 * (lane & 3)) =
+          ptx::pack_bf16x2(o_acc[nt][2 * hrow], o_acc[nt][2 * hrow + 1]);
     }
   }
-  __syncthreads();
-  if (trace && tid == 0) trace[4] = ptx::globaltimer();
-  cluster_wait();   // entry phase: every rank has started
-  if (trace && tid == 0) trace[5] = ptx::globaltimer();
-  // push every valid row (D bf16 = D*2 bytes) to the rank that combines it:
-  // one warp per row, 16 bytes per lane
+  __syncwarp();
+  const size_t part_base = (size_t)(g * a.Hq + j) * nchunk;   // partial slot of rank q: part_base + q
   {
-    const uint32_t rcv = ptx::smem_u32(recv), rml = ptx::smem_u32(recv_ml);
-    constexpr int CPRB = D / 8;   // 16-byte chunks per bf16 row
-    for (int r = warp; r < a.S; r += 8) {
-      const int owner = r / rpc, rl = r - owner * rpc;
-      const uint32_t dst = ptx::mapa(rcv, (uint32_t)owner) + (uint32_t)((rank * rpc + rl) * D * 2);
-      for (int ch = lane; ch < CPRB; ch += 32) {
-        const uint4 v = *reinterpret_cast<const uint4*>(ob_s + r * OS + ch * 8);
-        asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + (uint32_t)(ch * 16)), "r"(v.x),
-                     "r"(v.y), "r"(v.z), "r"(v.w)
-                     : "memory");
-      }
-      if (lane == 0) {
-        const uint32_t mdst = ptx::mapa(rml, (uint32_t)owner) + (uint32_t)((rank * rpc + rl) * 8);
-        asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(mdst), "f"(mml[r * 2]), "f"(mml[r * 2 + 1])
-                     : "memory");
-      }
+    __nv_bfloat16* po = a.part_o + (part_base + rank) * 64 * D;
+    for (int r = 16 * warp; r < min(a.S, 16 * warp + 16); ++r)
+      for (int ch = lane; ch < CPR; ch += 32)
+        *reinterpret_cast<uint4*>(po + (size_t)r * D + ch * 8) =
+            *reinterpret_cast<const uint4*>(Qs + r * D + ((ch ^ (r & 7)) << 3));
+    float* pml = a.part_ml + (part_base + rank) * 64 * 2;
+    if ((lane & 3) == 0) {
+      if (row0 < a.S) *reinterpret_cast<float2*>(pml + row0 * 2) = make_float2(m_r[0], l_r[0]);
+      if (row0 + 8 < a.S) *reinterpret_cast<float2*>(pml + (row0 + 8) * 2) = make_float2(m_r[1], l_r[1]);
     }
   }
-  if (trace && tid == 0) trace[6] = ptx::globaltimer();
+  if (trace && tid == 0) trace[4] = ptx::globaltimer();
+  // release / acquire at cluster scope: every rank's partials are visible
   ptx::cluster_sync();
-  if (trace && tid == 0) trace[7] = ptx::globaltimer();
-  // combine the ranks' partials for my rows, in rank order
-  const int r0 = rank * rpc, n_own = min(a.S, r0 + rpc) - r0;
-  if (tid < n_own) {
-    const int rl = tid;
-    float mx = -INFINITY;
-    for (int qr = 0; qr < nchunk; ++qr) mx = fmaxf(mx, recv_ml[(qr * rpc + rl) * 2]);
-    float lsum = 0.f;
-    for (int qr = 0; qr < nchunk; ++qr) {
-      const float mq = recv_ml[(qr * rpc + rl) * 2];
-      const float wq = mq == -INFINITY ? 0.f : exp2f(mq - mx);
-      wq_s[rl * nchunk + qr] = wq;
-      lsum = fmaf(wq, recv_ml[(qr * rpc + rl) * 2 + 1], lsum);
+  if (trace && tid == 0) trace[5] = trace[6] = trace[7] = ptx::globaltimer();
+  // combine: one warp per owned row; lane q < nchunk weighs rank q's partial,
+  // and the D outputs of the row are taken 8 per lane, ranks summed in order
+  const int r0 = rank * rpc, n_own = max(0, min(a.S, r0 + rpc) - r0);
+  for (int rl = warp; rl < n_own; rl += 4) {
+    const int r = r0 + rl;
+    float mq = -INFINITY, lq = 0.f;
+    if (lane < nchunk) {
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml + ((part_base + lane) * 64 + r) * 2));
+      mq = ml.x;
+      lq = ml.y;
     }
-    inv_s[rl] = 1.f / lsum;
-  }
-  __syncthreads();
-  for (int idx = tid; idx < n_own * (D / 2); idx += 256) {
-    const int rl = idx / (D / 2), d2 = idx - rl * (D / 2);
-    float ox = 0.f, oy = 0.f;
-    for (int qr = 0; qr < nchunk; ++qr) {
-      const float2 v = __bfloat1622float2(
-          *reinterpret_cast<const __nv_bfloat162*>(recv + (size_t)(qr * rpc + rl) * D + 2 * d2));
-      ox = fmaf(wq_s[rl * nchunk + qr], v.x, ox);
-      oy = fmaf(wq_s[rl * nchunk + qr], v.y, oy);
+    const float mx = warp_max(mq);
+    const float wq = (lane < nchunk && mq != -INFINITY) ? exp2f(mq - mx) : 0.f;
+    const float inv = 1.f / warp_sum(wq * lq);
+    for (int ch = lane; ch < CPR; ch += 32) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int q = 0; q < nchunk; ++q) {
+        const float wqq = __shfl_sync(0xffffffffu, wq, q);
+        const uint4 v = __ldcg(reinterpret_cast<const uint4*>(a.part_o + ((part_base + q) * 64 + r) * D + ch * 8));
+        const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(v2[e]);
+          acc[2 * e] = fmaf(wqq, f.x, acc[2 * e]);
+          acc[2 * e + 1] = fmaf(wqq, f.y, acc[2 * e + 1]);
+        }
+      }
+      uint4 out;
+      out.x = ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv);
+      out.y = ptx::pack_bf16x2(acc[2] * inv, acc[3] * inv);
+      out.z = ptx::pack_bf16x2(acc[4] * inv, acc[5] * inv);
+      out.w = ptx::pack_bf16x2(acc[6] * inv, acc[7] * inv);
+      *reinterpret_cast<uint4*>(a.o + ts_offset(g * a.S + r, j * D + ch * 8, a.n_mma)) = out;
     }
-    *reinterpret_cast<uint32_t*>(a.o + (((size_t)g * a.S + r0 + rl) * a.Hq + j) * D + 2 * d2) =
-        ptx::pack_bf16x2(ox * inv_s[rl], oy * inv_s[rl]);
   }
   if (trace && tid == 0) trace[8] = ptx::globaltimer();
 }
@@ -726,7 +722,7 @@ __global__ void __launch_bounds__(256) attn_mma_kernel(const AttnArgs a) {
 // ---------------------------------------------------------------------------
 struct StepArgs {
   float* h;                       // [T][w]
-  __nv_bfloat16* hb;              // [T][w]
+  __nv_bfloat16* hb;              // tiled [w/64][n_mma][64]
   float* ssp;                     // [T][w/128]
   float* x;                       // [G][H][A]
   float* vout;                    // [G][H][A] or nullptr
@@ -741,7 +737,7 @@ struct StepArgs {
   const float* b_sp;
   const float* g_attn0;           // first layer's attention-norm gain
   unsigned* status;
-  int w, S, A, Sd, state_stride, c_stride, do_head, do_embed;
+  int w, S, A, Sd, state_stride, c_stride, do_head, do_embed, n_mma;
   float dt, eps;
 };
 
@@ -841,7 +837,7 @@ __global__ void __launch_bounds__(256) step_kernel(const StepArgs a) {
   uint2 hbv;
   hbv.x = ptx::pack_bf16x2(hv[0] * (1.f + ga.x), hv[1] * (1.f + ga.y));
   hbv.y = ptx::pack_bf16x2(hv[2] * (1.f + ga.z), hv[3] * (1.f + ga.w));
-  *reinterpret_cast<uint2*>(a.hb + (size_t)r * a.w + i0) = hbv;
+  *reinterpret_cast<uint2*>(a.hb + ts_offset(r, i0, a.n_mma)) = hbv;
   // each warp covers one 128-feature tile
   float sq = hv[0] * hv[0];
   sq = fmaf(hv[1], hv[1], sq);
@@ -852,15 +848,18 @@ __global__ void __launch_bounds__(256) step_kernel(const StepArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Weight packing: gather rows of a [rows][K] bf16 matrix into a new order.
+// Weight packing: row r of the packed matrix is row idx[r] (or r) of a
+// [rows][K] bf16 matrix, stored in 128-row tiles of the tiled, pre-swizzled
+// layout ([rows/128][K/64][128][64], see ts_offset).
 // ---------------------------------------------------------------------------
-__global__ void gather_rows_kernel(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst,
-                                   const int* __restrict__ idx, int rows, int K) {
+__global__ void pack_tiled_kernel(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst,
+                                  const int* __restrict__ idx, int rows, int K) {
   const int r = blockIdx.x;
   if (r >= rows) return;
-  const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)idx[r] * K);
-  uint4* d = reinterpret_cast<uint4*>(dst + (size_t)r * K);
-  for (int i = threadIdx.x; i < K / 8; i += blockDim.x) d[i] = s[i];
+  const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)(idx ? idx[r] : r) * K);
+  __nv_bfloat16* d = dst + (size_t)(r >> 7) * (K >> 6) * 8192;
+  for (int i = threadIdx.x; i < K / 8; i += blockDim.x)
+    *reinterpret_cast<uint4*>(d + ts_offset(r & 127, 8 * i, 128)) = s[i];
 }
 
 // [rows][cols] -> [cols][rows]
@@ -883,13 +882,19 @@ struct GemmPlan {
 struct FastPath {
   __nv_bfloat16 *w_qkv = nullptr, *w_o = nullptr, *w_gu = nullptr, *w_down = nullptr;
   __nv_bfloat16 *w_aiT = nullptr, *w_spT = nullptr;
-  CUtensorMap map_qkv, map_o, map_gu, map_down;
   __nv_bfloat16 *qb = nullptr, *ksb = nullptr, *vsb = nullptr, *ob = nullptr, *mb = nullptr, *hb = nullptr;
   float* ssp = nullptr;
+  __nv_bfloat16* att_po = nullptr;   // attention partial rows [Gmax][Hq][16][64][D]
+  float* att_pml = nullptr;          // their (max, sum)       [Gmax][Hq][16][64][2]
   int num_sms = 148;
   int max_cluster = 8;
+  int gemm_fit_small[17] = {0};   // co-resident GEMM clusters by size, at the smem_cap budget (diagnostic)
+  int gemm_fit_large[17] = {0};   // ... and at the whole shared memory
   int attn_fit[17] = {0};      // co-resident clusters of attention CTAs, by cluster size
-  int smem_cap = 112 * 1024;   // keeps two CTAs per SM so the next kernel can prefetch
+  // Shared-memory budget of a GEMM grid larger than the SM count.  A kernel
+  // that holds tensor memory runs one CTA per SM whatever its shared memory;
+  // the budget leaves room beside it for a CTA of the attention or step kernel.
+  int smem_cap = 100 * 1024;
   // optional phase trace of the four projections of layer 0 in the first Euler step
   unsigned long long* trace = nullptr;
   int trace_ctas[5] = {0, 0, 0, 0, 0};
@@ -902,38 +907,12 @@ namespace {
 constexpr int kSmemOptin = 227 * 1024;
 constexpr int kDynSmemMax = kSmemOptin - 2048;   // every kernel here uses < 2 KB of static shared memory
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    cudaDriverEntryPointQueryResult q;
-    void* p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
-  }
-  return fn;
-}
-
-// 2-D row-major bf16 tensor [rows][K], box of 64 elements x box_rows rows, 128-byte swizzle.
-bool make_map(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t K, uint32_t box_rows) {
-  auto enc = get_encode();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {K, rows};
-  cuuint64_t strides[1] = {K * 2};
-  cuuint32_t box[2] = {64, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 // Split of one projection over CTAs: 128-row weight tiles x K slices (one
-// cluster per tile).  The smallest cluster that puts at least one CTA on
-// every SM is taken; the ring depth is then the largest that fits the
-// shared-memory budget.
+// cluster per tile, at most 8 CTAs).  The smallest cluster that puts at
+// least one CTA on every SM is taken; the ring depth is then the largest
+// that fits the shared-memory budget.
 GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T) {
   GemmPlan best;
   best.n_tiles = N / 128;
@@ -955,8 +934,7 @@ GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T) {
 }
 
 template <int MODE>
-cudaError_t launch_gemm(const CUtensorMap& map, const CUtensorMap& amap, const GemmArgs& a, const GemmPlan& pl,
-                        cudaStream_t st) {
+cudaError_t launch_gemm(const GemmArgs& a, const GemmPlan& pl, cudaStream_t st) {
   auto kern = gemm_tc_kernel<MODE>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.cs, pl.n_tiles, 1);
@@ -975,7 +953,7 @@ cudaError_t launch_gemm(const CUtensorMap& map, const CUtensorMap& amap, const G
   GemmArgs args = a;
   args.kslice = pl.kslice;
   args.stages = pl.stages;
-  return cudaLaunchKernelEx(&cfg, kern, map, amap, args);
+  return cudaLaunchKernelEx(&cfg, kern, args);
 }
 
 // Dynamic shared memory a kernel may request: the per-block opt-in limit
@@ -1009,8 +987,8 @@ template <int D>
 int attn_clusters_that_fit(int cs, int S) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs, 1, 1);
-  cfg.blockDim = dim3(256, 1, 1);
-  cfg.dynamicSmemBytes = attn_smem_bytes(D, cs, (S + cs - 1) / cs);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = attn_smem_bytes(D);
   cudaLaunchAttribute at;
   at.id = cudaLaunchAttributeClusterDimension;
   at.val.clusterDim.x = cs;
@@ -1029,8 +1007,8 @@ cudaError_t launch_attn(const AttnArgs& a, int nchunk, int G, cudaStream_t st) {
   auto kern = attn_mma_kernel<D>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nchunk, a.Hq, G);
-  cfg.blockDim = dim3(256, 1, 1);
-  cfg.dynamicSmemBytes = attn_smem_bytes(D, nchunk, (a.S + nchunk - 1) / nchunk);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = attn_smem_bytes(D);
   cfg.stream = st;
   cudaLaunchAttribute attrs[2];
   attrs[0].id = cudaLaunchAttributeClusterDimension;
@@ -1079,7 +1057,7 @@ rtv_status fast_create(rtv_ctx* ctx) {
   const int n_mma_max = round_up(ctx->Gmax * S, 16);
   const bool shape_ok = k.dtype == RTV_BF16 && (k.head_dim == 128 || k.head_dim == 256) && k.width % 128 == 0 &&
                         k.width <= 1024 && k.mlp_dim % 128 == 0 && (ctx->Q % 128) == 0 && S <= 64 &&
-                        k.action_dim <= 64 && k.state_dim <= 64 && n_mma_max <= 256 && get_encode() != nullptr;
+                        k.action_dim <= 64 && k.state_dim <= 64 && n_mma_max <= 256;
   if (!shape_ok) return RTV_OK;
   int dev = ctx->device;
   if (configure_gemm<GM_QKV>() != cudaSuccess || configure_gemm<GM_O>() != cudaSuccess ||
@@ -1090,35 +1068,41 @@ rtv_status fast_create(rtv_ctx* ctx) {
   }
   FastPath* fp = new FastPath();
   cudaDeviceGetAttribute(&fp->num_sms, cudaDevAttrMultiProcessorCount, dev);
-  // largest cluster that can be co-scheduled for the GEMM kernel
-  {
-    auto kern = gemm_tc_kernel<GM_DOWN>;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(16, 8, 1);
-    cfg.blockDim = dim3(192, 1, 1);
-    cfg.dynamicSmemBytes = 100 * 1024;
-    cudaLaunchAttribute at;
-    at.id = cudaLaunchAttributeClusterDimension;
-    at.val.clusterDim.x = 16;
-    at.val.clusterDim.y = 1;
-    at.val.clusterDim.z = 1;
-    cfg.attrs = &at;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n >= 8) fp->max_cluster = 16;
-    cudaGetLastError();
+  // co-resident GEMM clusters by cluster size, at both shared-memory budgets
+  for (int cs = 1; cs <= 16; cs <<= 1) {
+    for (int big = 0; big < 2; ++big) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(cs, 1, 1);
+      cfg.blockDim = dim3(192, 1, 1);
+      cfg.dynamicSmemBytes = big ? kDynSmemMax : fp->smem_cap;
+      cudaLaunchAttribute at;
+      at.id = cudaLaunchAttributeClusterDimension;
+      at.val.clusterDim.x = cs;
+      at.val.clusterDim.y = 1;
+      at.val.clusterDim.z = 1;
+      cfg.attrs = &at;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<GM_DOWN>, &cfg) != cudaSuccess) n = 0;
+      cudaGetLastError();
+      (big ? fp->gemm_fit_large : fp->gemm_fit_small)[cs] = n;
+    }
   }
+  fp->max_cluster = 8;
   for (int c : {2, 4, 6, 8, 12, 16})
     fp->attn_fit[c] = k.head_dim == 256 ? attn_clusters_that_fit<256>(c, S) : attn_clusters_that_fit<128>(c, S);
   const size_t T = ctx->Tmax;
+  const size_t Tp = (size_t)round_up(ctx->Tmax, 16);   // token rows of the tiled GEMM inputs
   auto alloc = [&](void** p, size_t bytes) -> bool {
     if (cudaMalloc(p, bytes) != cudaSuccess) return false;
     fp->allocs.push_back(*p);
-    return true;
+    return cudaMemset(*p, 0, bytes) == cudaSuccess;
   };
-  bool ok = alloc((void**)&fp->qb, T * ctx->Q * 2) && alloc((void**)&fp->ob, T * ctx->Q * 2) &&
-            alloc((void**)&fp->mb, T * (size_t)k.mlp_dim * 2) && alloc((void**)&fp->hb, T * (size_t)k.width * 2) &&
+  bool ok = alloc((void**)&fp->qb, T * ctx->Q * 2) && alloc((void**)&fp->ob, Tp * ctx->Q * 2) &&
+            alloc((void**)&fp->mb, Tp * (size_t)k.mlp_dim * 2) && alloc((void**)&fp->hb, Tp * (size_t)k.width * 2) &&
             alloc((void**)&fp->ssp, T * (size_t)(k.width / 128) * 4) &&
+            alloc((void**)&fp->att_po, (size_t)ctx->Gmax * k.n_q_heads * 16 * 64 * k.head_dim * 2) &&
+            alloc((void**)&fp->att_pml, (size_t)ctx->Gmax * k.n_q_heads * 16 * 64 * 2 * 4) &&
             alloc((void**)&fp->ksb, (size_t)ctx->Gmax * ctx->KV * S * 2) &&
             alloc((void**)&fp->vsb, (size_t)ctx->Gmax * ctx->KV * S * 2);
   if (!ok) {
@@ -1127,9 +1111,9 @@ rtv_status fast_create(rtv_ctx* ctx) {
     return RTV_ERR_OOM;
   }
   if (getenv("RTV_TRACE")) {
-    if (cudaMalloc(&fp->trace, 5 * 512 * 16 * sizeof(unsigned long long)) == cudaSuccess) {
+    if (cudaMalloc(&fp->trace, 5 * 512 * kTraceRow * sizeof(unsigned long long)) == cudaSuccess) {
       fp->allocs.push_back(fp->trace);
-      cudaMemset(fp->trace, 0, 5 * 512 * 16 * sizeof(unsigned long long));
+      cudaMemset(fp->trace, 0, 5 * 512 * kTraceRow * sizeof(unsigned long long));
     } else {
       fp->trace = nullptr;
     }
@@ -1147,35 +1131,49 @@ void fast_arm_trace(rtv_ctx* ctx) {
 void fast_trace_report(rtv_ctx* ctx) {
   FastPath* fp = ctx->fast;
   if (!fp || !fp->trace || !fp->trace_ctas[0]) return;
-  std::vector<unsigned long long> h(5 * 512 * 16);
+  std::vector<unsigned long long> h(5 * 512 * kTraceRow);
   cudaDeviceSynchronize();
   cudaMemcpy(h.data(), fp->trace, h.size() * 8, cudaMemcpyDeviceToHost);
   const char* nm[5] = {"qkv", "o", "gu", "down", "attention"};
-  const char* ev[2][13] = {{"start", "w_issued", "pdl", "first_full", "mma_issued", "done", "copied", "recv", "end",
-                           "prefetched", "arrived", "iter0", "exit"},
+  const char* ev[2][15] = {{"start", "w_issued", "pdl", "first_full", "mma_issued", "done", "copied", "recv", "end",
+                           "prefetched", "arrived", "iter0", "exit", "part", "entry"},
                           {"start", "pdl", "tile0", "loop_end", "merged", "entry", "pushed", "synced", "end", "", "", "",
-                           ""}};
+                           "", "", ""}};
   unsigned long long t_ref = ~0ull;
   for (int i = 0; i < 5; ++i)
     for (int c = 0; c < fp->trace_ctas[i]; ++c)
-      if (h[((size_t)i * 512 + c) * 16]) t_ref = std::min(t_ref, h[((size_t)i * 512 + c) * 16]);
+      if (h[((size_t)i * 512 + c) * kTraceRow]) t_ref = std::min(t_ref, h[((size_t)i * 512 + c) * kTraceRow]);
   const int order[5] = {0, 4, 1, 2, 3};
   for (int oi = 0; oi < 5; ++oi) {
     const int i = order[oi];
     fprintf(stderr, "[rtv trace] %s (%d CTAs), us after the first traced start: min / median / max\n", nm[i],
             fp->trace_ctas[i]);
-    const int order_e[13] = {0, 1, 2, 3, 4, 5, 6, 9, 7, 10, 11, 8, 12};
-    for (int ei = 0; ei < 13; ++ei) {
+    const int order_e[15] = {0, 1, 2, 3, 4, 5, 13, 14, 6, 9, 7, 10, 11, 8, 12};
+    for (int ei = 0; ei < 15; ++ei) {
       const int e = order_e[ei];
       if (!ev[i == 4][e][0]) continue;
       std::vector<double> v;
       for (int c = 0; c < fp->trace_ctas[i]; ++c) {
-        const unsigned long long t = h[((size_t)i * 512 + c) * 16 + e];
+        const unsigned long long t = h[((size_t)i * 512 + c) * kTraceRow + e];
         if (t) v.push_back((double)(t - t_ref) * 1e-3);
       }
       if (v.empty()) continue;
       std::sort(v.begin(), v.end());
       fprintf(stderr, "    %-11s %8.2f %8.2f %8.2f\n", ev[i == 4][e], v.front(), v[v.size() / 2], v.back());
+    }
+    if (i != 4) {
+      fprintf(stderr, "    stage landed (median):");
+      for (int b = 0; b < 8; ++b) {
+        std::vector<double> v;
+        for (int c = 0; c < fp->trace_ctas[i]; ++c) {
+          const unsigned long long t = h[((size_t)i * 512 + c) * kTraceRow + 16 + b];
+          if (t) v.push_back((double)(t - t_ref) * 1e-3);
+        }
+        if (v.empty()) break;
+        std::sort(v.begin(), v.end());
+        fprintf(stderr, " %.2f", v[v.size() / 2]);
+      }
+      fprintf(stderr, "\n");
     }
   }
 }
@@ -1214,12 +1212,12 @@ rtv_status fast_load(rtv_ctx* ctx, const rtv_tensor*, int) {
   cudaMemcpy(d_igu, igu.data(), ngu * 4, cudaMemcpyHostToDevice);
   for (int l = 0; l < Lh; ++l) {
     const LayerW& Lw = ctx->W.layers[l];
-    gather_rows_kernel<<<(int)nq, 128>>>((const __nv_bfloat16*)Lw.qkv, fp->w_qkv + (size_t)l * nq * w, d_iq,
-                                         (int)nq, w);
-    gather_rows_kernel<<<(int)ngu, 128>>>((const __nv_bfloat16*)Lw.gu, fp->w_gu + (size_t)l * ngu * w, d_igu,
-                                          (int)ngu, w);
-    cudaMemcpy(fp->w_o + (size_t)l * w * Q, Lw.o, (size_t)w * Q * 2, cudaMemcpyDeviceToDevice);
-    cudaMemcpy(fp->w_down + (size_t)l * w * F, Lw.down, (size_t)w * F * 2, cudaMemcpyDeviceToDevice);
+    pack_tiled_kernel<<<(int)nq, 128>>>((const __nv_bfloat16*)Lw.qkv, fp->w_qkv + (size_t)l * nq * w, d_iq,
+                                        (int)nq, w);
+    pack_tiled_kernel<<<(int)ngu, 128>>>((const __nv_bfloat16*)Lw.gu, fp->w_gu + (size_t)l * ngu * w, d_igu,
+                                         (int)ngu, w);
+    pack_tiled_kernel<<<w, 128>>>((const __nv_bfloat16*)Lw.o, fp->w_o + (size_t)l * w * Q, nullptr, w, Q);
+    pack_tiled_kernel<<<w, 128>>>((const __nv_bfloat16*)Lw.down, fp->w_down + (size_t)l * w * F, nullptr, w, F);
   }
   transpose_bf16_kernel<<<64, 256>>>((const __nv_bfloat16*)ctx->W.ai_w, fp->w_aiT, w, k.action_dim);
   transpose_bf16_kernel<<<64, 256>>>((const __nv_bfloat16*)ctx->W.sp_w, fp->w_spT, w, k.state_dim);
@@ -1227,10 +1225,6 @@ rtv_status fast_load(rtv_ctx* ctx, const rtv_tensor*, int) {
   cudaFree(d_iq);
   cudaFree(d_igu);
   if (e != cudaSuccess) return RTV_ERR_CUDA;
-  if (!make_map(&fp->map_qkv, fp->w_qkv, Lh * nq, w, 128) || !make_map(&fp->map_o, fp->w_o, (size_t)Lh * w, Q, 128) ||
-      !make_map(&fp->map_gu, fp->w_gu, Lh * ngu, w, 128) ||
-      !make_map(&fp->map_down, fp->w_down, (size_t)Lh * w, F, 128))
-    return RTV_ERR_CUDA;
   return RTV_OK;
 }
 
@@ -1265,6 +1259,7 @@ rtv_status fast_step(rtv_ctx* ctx, int G, bool do_head, bool do_embed, float dt,
   a.do_embed = do_embed ? 1 : 0;
   a.dt = dt;
   a.eps = k.rms_eps;
+  a.n_mma = round_up(G * ctx->S, 16);
   const cudaError_t e = launch_step(a, G * ctx->S, st);
   if (e != cudaSuccess) {
     ctx->last_error = std::string("step launch: ") + cudaGetErrorString(e);
@@ -1287,16 +1282,9 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
   const int nk = P + S;
   const int nchunk = attn_chunks(fp, nk, k.n_q_heads * G);
   if (!(p_qkv.valid && p_o.valid && p_gu.valid && p_dn.valid) ||
-      attn_smem_bytes(D, nchunk, (S + nchunk - 1) / nchunk) > kDynSmemMax) {
+      attn_smem_bytes(D) > kDynSmemMax || nchunk > 16) {
     ctx->last_error = "no tensor-core split fits this token count";
     return RTV_ERR_UNSUPPORTED;
-  }
-  // activation tensor maps for this token count (rows beyond T read as zeros)
-  CUtensorMap m_h, m_o, m_m;
-  if (!make_map(&m_h, fp->hb, T, w, n_mma) || !make_map(&m_o, fp->ob, T, Q, n_mma) ||
-      !make_map(&m_m, fp->mb, T, F, n_mma)) {
-    ctx->last_error = "activation tensor map encoding failed";
-    return RTV_ERR_CUDA;
   }
   if (getenv("RTV_LOG")) {
     const GemmPlan* pls[4] = {&p_qkv, &p_o, &p_gu, &p_dn};
@@ -1304,8 +1292,11 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     for (int i = 0; i < 4; ++i)
       fprintf(stderr, "[rtv] T=%d %s: tiles=%d cluster=%d kslice=%d stages=%d smem=%d\n", T, nm[i], pls[i]->n_tiles,
               pls[i]->cs, pls[i]->kslice, pls[i]->stages, pls[i]->smem);
+    fprintf(stderr, "[rtv] gemm clusters that fit (size: two-per-SM budget / whole smem):");
+    for (int cs = 1; cs <= 16; cs <<= 1) fprintf(stderr, " %d: %d/%d", cs, fp->gemm_fit_small[cs], fp->gemm_fit_large[cs]);
+    fprintf(stderr, "\n");
     fprintf(stderr, "[rtv] attention: chunks=%d keys/chunk=%d smem=%d max_cluster=%d sms=%d fit(8,12,16)=%d,%d,%d\n",
-            nchunk, (nk + nchunk - 1) / nchunk, attn_smem_bytes(D, nchunk, (S + nchunk - 1) / nchunk), fp->max_cluster,
+            nchunk, (nk + nchunk - 1) / nchunk, attn_smem_bytes(D), fp->max_cluster,
             fp->num_sms, fp->attn_fit[8], fp->attn_fit[12], fp->attn_fit[16]);
   }
 
@@ -1336,6 +1327,8 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
   at.sk = fp->ksb;
   at.sv = fp->vsb;
   at.o = fp->ob;
+  at.part_o = fp->att_po;
+  at.part_ml = fp->att_pml;
   at.status = ctx->status;
   at.S = S;
   at.P = P;
@@ -1345,6 +1338,7 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
   at.pbs = prefix_batch_stride;
   at.mask_mode = k.suffix_mask;
   at.kpc = (nk + nchunk - 1) / nchunk;
+  at.n_mma = n_mma;
   at.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
   const size_t kv_layer = (size_t)k.max_batch * k.n_kv_heads * k.max_prefix_len * D;
 
@@ -1358,15 +1352,18 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     fp->trace_ctas[4] = nchunk * k.n_q_heads * G;
   }
   auto tr = [&](int l, int i) -> unsigned long long* {
-    return (tracing && l == 0) ? fp->trace + (size_t)i * 512 * 16 : nullptr;
+    return (tracing && l == 0) ? fp->trace + (size_t)i * 512 * kTraceRow : nullptr;
   };
 
   for (int l = 0; l < k.n_layers; ++l) {
     const LayerW& Lw = ctx->W.layers[l];
     GemmArgs a = base;
     a.trace = tr(l, 0);
-    a.w_row0 = l * nq;
-    cudaError_t e = launch_gemm<GM_QKV>(fp->map_qkv, m_h, a, p_qkv, st);
+    a.wt = fp->w_qkv;
+    a.act = fp->hb;
+    a.K = w;
+    a.w_tile0 = l * nq / 128;
+    cudaError_t e = launch_gemm<GM_QKV>(a, p_qkv, st);
 
     at.trace = tr(l, 4);
     at.pk = (const __nv_bfloat16*)ctx->prefix_kv + (size_t)(2 * l) * kv_layer;
@@ -1375,20 +1372,29 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
 
     a = base;
     a.trace = tr(l, 1);
-    a.w_row0 = l * w;
+    a.wt = fp->w_o;
+    a.act = fp->ob;
+    a.K = Q;
+    a.w_tile0 = l * w / 128;
     a.g_next = Lw.g_mlp;
-    if (e == cudaSuccess) e = launch_gemm<GM_O>(fp->map_o, m_o, a, p_o, st);
+    if (e == cudaSuccess) e = launch_gemm<GM_O>(a, p_o, st);
 
     a = base;
     a.trace = tr(l, 2);
-    a.w_row0 = l * 2 * F;
-    if (e == cudaSuccess) e = launch_gemm<GM_GU>(fp->map_gu, m_h, a, p_gu, st);
+    a.wt = fp->w_gu;
+    a.act = fp->hb;
+    a.K = w;
+    a.w_tile0 = l * 2 * F / 128;
+    if (e == cudaSuccess) e = launch_gemm<GM_GU>(a, p_gu, st);
 
     a = base;
     a.trace = tr(l, 3);
-    a.w_row0 = l * w;
+    a.wt = fp->w_down;
+    a.act = fp->mb;
+    a.K = F;
+    a.w_tile0 = l * w / 128;
     a.g_next = (l + 1 < k.n_layers) ? ctx->W.layers[l + 1].g_attn : nullptr;
-    if (e == cudaSuccess) e = launch_gemm<GM_DOWN>(fp->map_down, m_m, a, p_dn, st);
+    if (e == cudaSuccess) e = launch_gemm<GM_DOWN>(a, p_dn, st);
     if (e != cudaSuccess) {
       ctx->last_error = std::string("tensor-core launch: ") + cudaGetErrorString(e);
       return RTV_ERR_CUDA;
