@@ -478,7 +478,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
   const int nchunk = gridDim.x;
   const int rpc = (a.S + nchunk - 1) / nchunk;   // query rows combined by each rank
   // every CTA of the grid sees the same values, so a refusal is uniform
-  if (dynamic_smem_size() < (uint32_t)attn_smem_bytes(D) || a.S > 64 || nchunk > 32) {
+  if (dynamic_smem_size() < (uint32_t)attn_smem_bytes(D) || a.S > 64 || nchunk > 16) {
     if (threadIdx.x == 0) atomicOr(a.status, RTV_DEV_BOUNDS);
     return;
   }
@@ -672,7 +672,8 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
   ptx::cluster_sync();
   if (trace && tid == 0) trace[5] = trace[6] = trace[7] = ptx::globaltimer();
   // combine: one warp per owned row; lane q < nchunk weighs rank q's partial,
-  // and the D outputs of the row are taken 8 per lane, ranks summed in order
+  // and the D outputs of the row are taken 8 per lane, ranks summed in order.
+  // All of a lane's loads are issued before any is used.
   const int r0 = rank * rpc, n_own = max(0, min(a.S, r0 + rpc) - r0);
   for (int rl = warp; rl < n_own; rl += 4) {
     const int r = r0 + rl;
@@ -682,28 +683,38 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
       mq = ml.x;
       lq = ml.y;
     }
-    const float mx = warp_max(mq);
-    const float wq = (lane < nchunk && mq != -INFINITY) ? exp2f(mq - mx) : 0.f;
-    const float inv = 1.f / warp_sum(wq * lq);
-    for (int ch = lane; ch < CPR; ch += 32) {
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int q = 0; q < nchunk; ++q) {
-        const float wqq = __shfl_sync(0xffffffffu, wq, q);
-        const uint4 v = __ldcg(reinterpret_cast<const uint4*>(a.part_o + ((part_base + q) * 64 + r) * D + ch * 8));
-        const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+    for (int ch0 = 0; ch0 < CPR; ch0 += 32) {
+      const int ch = ch0 + lane;
+      uint4 v[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __bfloat1622float2(v2[e]);
-          acc[2 * e] = fmaf(wqq, f.x, acc[2 * e]);
-          acc[2 * e + 1] = fmaf(wqq, f.y, acc[2 * e + 1]);
+      for (int q = 0; q < 16; ++q)
+        if (q < nchunk && ch < CPR)
+          v[q] = __ldcg(reinterpret_cast<const uint4*>(a.part_o + ((part_base + q) * 64 + r) * D + ch * 8));
+      const float mx = warp_max(mq);
+      const float wq = (lane < nchunk && mq != -INFINITY) ? exp2f(mq - mx) : 0.f;
+      const float inv = 1.f / warp_sum(wq * lq);
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const float wqq = __shfl_sync(0xffffffffu, wq, q);
+        if (q < nchunk && ch < CPR) {
+          const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&v[q]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(v2[e]);
+            acc[2 * e] = fmaf(wqq, f.x, acc[2 * e]);
+            acc[2 * e + 1] = fmaf(wqq, f.y, acc[2 * e + 1]);
+          }
         }
       }
-      uint4 out;
-      out.x = ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv);
-      out.y = ptx::pack_bf16x2(acc[2] * inv, acc[3] * inv);
-      out.z = ptx::pack_bf16x2(acc[4] * inv, acc[5] * inv);
-      out.w = ptx::pack_bf16x2(acc[6] * inv, acc[7] * inv);
-      *reinterpret_cast<uint4*>(a.o + ts_offset(g * a.S + r, j * D + ch * 8, a.n_mma)) = out;
+      if (ch < CPR) {
+        uint4 out;
+        out.x = ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv);
+        out.y = ptx::pack_bf16x2(acc[2] * inv, acc[3] * inv);
+        out.z = ptx::pack_bf16x2(acc[4] * inv, acc[5] * inv);
+        out.w = ptx::pack_bf16x2(acc[6] * inv, acc[7] * inv);
+        *reinterpret_cast<uint4*>(a.o + ts_offset(g * a.S + r, j * D + ch * 8, a.n_mma)) = out;
+      }
     }
   }
   if (trace && tid == 0) trace[8] = ptx::globaltimer();
