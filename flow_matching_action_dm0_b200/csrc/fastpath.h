@@ -15,6 +15,8 @@ rtv_status fast_create(rtv_ctx* ctx);
 // Pack the loaded parameters into the tensor-core layouts.
 rtv_status fast_load(rtv_ctx* ctx, const rtv_tensor* params, int n_params);
 bool fast_supports_prefix(rtv_ctx* ctx, int prefix_len);
+// Refresh the tensor-core layouts of the cached prefix after ctx->prefix_kv changed.
+rtv_status fast_prefix_update(rtv_ctx* ctx, int batch, int prefix_len, cudaStream_t st);
 // Step boundary over G suffixes: output head (Euler update of ctx->x, or the
 // velocity into ctx->v when velocity_only) and/or the suffix embedding of the
 // next evaluation into ctx->h with time condition rows c (stride c_stride).

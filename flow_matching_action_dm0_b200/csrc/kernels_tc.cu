@@ -77,6 +77,10 @@ struct GemmArgs {
   __nv_bfloat16* q;           // [T][Hq][D]
   __nv_bfloat16* ks;          // suffix keys   [G][Hkv][S][D]
   __nv_bfloat16* vs;          // suffix values [G][Hkv][S][D]
+  // When qt is set, q/k/v go instead to the tensor-core attention's tiles:
+  __nv_bfloat16* qt;          // q of head pairs [G][Hq/2][128 rows = 2 heads x 64][D], tiled (ts_offset, 128 rows)
+  __nv_bfloat16* kts;         // suffix keys [G][Hkv][64][D], tiled (64 rows)
+  __nv_bfloat16* vts;         // suffix values transposed [G][Hkv][D][64], tiled (D rows, 64 keys)
   const float* rope_cs;       // [S][D/2]
   const float* rope_sn;
   __nv_bfloat16* m;           // gelu(gate) * up, tiled [F/64][n_mma][64]
@@ -412,12 +416,32 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const GemmArgs a) {
             y1 = make_float2(x1.x * c.x - x2.x * sn.x, x1.y * c.y - x2.y * sn.y);
             y2 = make_float2(x2.x * c.x + x1.x * sn.x, x2.y * c.y + x1.y * sn.y);
           }
-          __nv_bfloat16* dst;
-          if (hh < a.Hq) dst = a.q + ((size_t)t * a.Hq + hh) * a.D;
-          else if (hh < a.Hq + a.Hkv) dst = a.ks + (((size_t)g * a.Hkv + (hh - a.Hq)) * a.S + s) * a.D;
-          else dst = a.vs + (((size_t)g * a.Hkv + (hh - a.Hq - a.Hkv)) * a.S + s) * a.D;
-          *reinterpret_cast<uint32_t*>(dst + dq0 + f0) = ptx::pack_bf16x2(y1.x, y1.y);
-          *reinterpret_cast<uint32_t*>(dst + dq0 + f0 + hd) = ptx::pack_bf16x2(y2.x, y2.y);
+          const int d1 = dq0 + f0, d2 = d1 + hd;
+          if (a.qt) {
+            if (hh < a.Hq) {
+              __nv_bfloat16* dst = a.qt + (size_t)(g * (a.Hq >> 1) + (hh >> 1)) * 128 * a.D;
+              const int row = ((hh & 1) << 6) + s;
+              *reinterpret_cast<uint32_t*>(dst + ts_offset(row, d1, 128)) = ptx::pack_bf16x2(y1.x, y1.y);
+              *reinterpret_cast<uint32_t*>(dst + ts_offset(row, d2, 128)) = ptx::pack_bf16x2(y2.x, y2.y);
+            } else if (hh < a.Hq + a.Hkv) {
+              __nv_bfloat16* dst = a.kts + (size_t)(g * a.Hkv + (hh - a.Hq)) * 64 * a.D;
+              *reinterpret_cast<uint32_t*>(dst + ts_offset(s, d1, 64)) = ptx::pack_bf16x2(y1.x, y1.y);
+              *reinterpret_cast<uint32_t*>(dst + ts_offset(s, d2, 64)) = ptx::pack_bf16x2(y2.x, y2.y);
+            } else {
+              __nv_bfloat16* dst = a.vts + (size_t)(g * a.Hkv + (hh - a.Hq - a.Hkv)) * a.D * 64;
+              dst[ts_offset(d1, s, a.D)] = __float2bfloat16_rn(y1.x);
+              dst[ts_offset(d1 + 1, s, a.D)] = __float2bfloat16_rn(y1.y);
+              dst[ts_offset(d2, s, a.D)] = __float2bfloat16_rn(y2.x);
+              dst[ts_offset(d2 + 1, s, a.D)] = __float2bfloat16_rn(y2.y);
+            }
+          } else {
+            __nv_bfloat16* dst;
+            if (hh < a.Hq) dst = a.q + ((size_t)t * a.Hq + hh) * a.D;
+            else if (hh < a.Hq + a.Hkv) dst = a.ks + (((size_t)g * a.Hkv + (hh - a.Hq)) * a.S + s) * a.D;
+            else dst = a.vs + (((size_t)g * a.Hkv + (hh - a.Hq - a.Hkv)) * a.S + s) * a.D;
+            *reinterpret_cast<uint32_t*>(dst + d1) = ptx::pack_bf16x2(y1.x, y1.y);
+            *reinterpret_cast<uint32_t*>(dst + d2) = ptx::pack_bf16x2(y2.x, y2.y);
+          }
         }
       }
       if (trace && tid == 0 && tl == 0) trace[TR_ITER0] = ptx::globaltimer();
@@ -721,6 +745,335 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Attention on the tensor cores, for head pairs that share a KV head
+// ("DM0.5 reading guide", sec. 5.1-5.2; same computation as the kernel above).
+// A cluster owns one (head pair, suffix); rank c takes key tile c of
+// [prefix tiles of 64 keys ; the suffix tile].  Rows are the 2 x 64 query
+// rows of the pair (rows past the suffix length are padding).
+//   S = Q K^T         tcgen05, M = 128 rows, N = 64 keys, K = D  -> TMEM
+//   P = exp2(S - max)  one thread per row, straight from TMEM, P -> shared memory (bf16)
+//   O = P V            tcgen05, M = 128, N = D, K = 64 keys, with V^T as the K-major operand -> TMEM
+// Each rank writes its unnormalised O rows and (max, sum) to global memory,
+// the cluster synchronises, and every rank combines the rows it owns, in
+// rank order, as in the kernel above.  Q, K and V^T arrive as tiled,
+// pre-swizzled blocks (ts_offset), one bulk copy each; the prefix tiles are
+// requested before waiting on the previous kernel.
+// ---------------------------------------------------------------------------
+struct AttnTcArgs {
+  const __nv_bfloat16* qt;    // [G][Hq/2][128][D] tiled
+  const __nv_bfloat16* pkt;   // this layer's prefix key tiles   [Bmax][Hkv][ntile_max][64][D]
+  const __nv_bfloat16* pvt;   // this layer's prefix value tiles [Bmax][Hkv][ntile_max][D][64] (transposed)
+  const __nv_bfloat16* kts;   // suffix key tiles   [G][Hkv][64][D]
+  const __nv_bfloat16* vts;   // suffix value tiles [G][Hkv][D][64]
+  __nv_bfloat16* o;           // attention output, tiled [Hq*D/64][n_mma][64]
+  __nv_bfloat16* part_o;      // partial rows [G][Hq/2][nchunk][128][D] (scratch)
+  float* part_ml;             // their (max, sum) [G][Hq/2][nchunk][128][2]
+  unsigned* status;
+  unsigned long long* trace;  // optional phase stamps [cta][kTraceRow], or nullptr
+  long long timeout_ns;
+  int S, P, Hq, Hkv, pbs, mask_mode, ntile_max, n_mma;
+  float scale_log2;
+};
+
+__host__ __device__ inline int attn_tc_smem_bytes(int D) { return 128 * D * 2 + 2 * 64 * D * 2 + 128 * 128 + 64 + 1024; }
+
+template <int D>
+__global__ void __launch_bounds__(256, 1) attn_tc_kernel(const AttnTcArgs a) {
+  extern __shared__ uint8_t sm_atc[];
+  __shared__ float red_m[2][128], red_l[2][128];   // per-row partial max / sum of the two column halves
+  constexpr int QB = 128 * D * 2, KB = 64 * D * 2, VB = D * 64 * 2, PB = 128 * 128;
+  // Tensor memory: S in columns [0, 64), then O in columns [0, D) -- the PV
+  // MMA is issued only after every thread has read S.  At most D <= 256
+  // columns, so this CTA and any GEMM CTA sharing its SM (at most 256
+  // columns each, and shared memory admits no third) never exceed the 512
+  // columns: no allocation ever waits on a CTA of a later kernel.
+  constexpr uint32_t TCOLS = D;
+  constexpr int CPR = D / 8;
+  const int nch = gridDim.x;
+  const int ntp = (a.P + 63) / 64;   // prefix tiles; rank ntp holds the suffix tile
+  // every CTA of the grid sees the same values, so a refusal is uniform
+  if (dynamic_smem_size() < (uint32_t)attn_tc_smem_bytes(D) || a.S > 64 || nch != ntp + 1 || nch > 16 ||
+      ntp > a.ntile_max) {
+    if (threadIdx.x == 0) atomicOr(a.status, RTV_DEV_BOUNDS);
+    return;
+  }
+  uint8_t* Qs = (uint8_t*)(((uintptr_t)sm_atc + 1023) & ~(uintptr_t)1023);
+  uint8_t* Ks = Qs + QB;
+  uint8_t* Vs = Ks + KB;
+  uint8_t* Ps = Vs + VB;
+  uint64_t* bars = (uint64_t*)(Ps + PB);   // 0: K and V^T landed, 1: Q landed, 2: S done, 3: O done
+  uint32_t* tslot = (uint32_t*)(bars + 4);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // warps w and w + 4 share TMEM lanes 32(w%4).. (rows) and split the columns
+  const int quarter = warp & 3, half = warp >> 2;
+  const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+  const int rank = (int)ptx::cluster_ctarank();
+  const int hp = blockIdx.y, g = blockIdx.z;
+  const int HP = a.Hq >> 1;
+  const int kvh = (2 * hp * a.Hkv) / a.Hq;
+  const bool suffix_tile = rank == ntp;
+  unsigned long long* trace =
+      a.trace ? a.trace + (((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * kTraceRow
+              : nullptr;
+  if (trace && tid == 0) trace[0] = ptx::globaltimer();
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) ptx::mbar_init(&bars[i], 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0) {
+    ptx::tmem_alloc(tslot, TCOLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tslot;
+  ptx::pdl_launch_dependents();
+  // the cached prefix does not depend on the previous kernel
+  if (tid == 0 && !suffix_tile) {
+    const size_t tile = ((size_t)(g * a.pbs) * a.Hkv + kvh) * a.ntile_max + rank;
+    ptx::mbar_expect_tx(&bars[0], (uint32_t)(KB + VB));
+    ptx::bulk_load(Ks, a.pkt + tile * 64 * D, (uint32_t)KB, &bars[0]);
+    ptx::bulk_load(Vs, a.pvt + tile * 64 * D, (uint32_t)VB, &bars[0]);
+  }
+  ptx::pdl_wait();
+  if (trace && tid == 0) trace[1] = ptx::globaltimer();
+  bool ok = true;
+  if (tid == 0) {
+    if (suffix_tile) {
+      const size_t tile = (size_t)g * a.Hkv + kvh;
+      ptx::mbar_expect_tx(&bars[0], (uint32_t)(KB + VB));
+      ptx::bulk_load(Ks, a.kts + tile * 64 * D, (uint32_t)KB, &bars[0]);
+      ptx::bulk_load(Vs, a.vts + tile * 64 * D, (uint32_t)VB, &bars[0]);
+    }
+    ptx::mbar_expect_tx(&bars[1], (uint32_t)QB);
+    const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(a.qt + (size_t)(g * HP + hp) * 128 * D);
+    for (int c = 0; c < QB; c += 16384) ptx::bulk_load(Qs + c, qsrc + c, 16384u, &bars[1]);
+    ok = ptx::mbar_wait(&bars[1], 0, a.timeout_ns) && ptx::mbar_wait(&bars[0], 0, a.timeout_ns);
+    if (ok) {
+      if (trace) trace[2] = ptx::globaltimer();
+      ptx::tc_fence_after();
+      const uint32_t idesc = ptx::idesc_bf16_f32(128, 64);
+      const uint32_t qa = ptx::smem_u32(Qs), ka = ptx::smem_u32(Ks);
+#pragma unroll
+      for (int kb = 0; kb < D / 64; ++kb)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::umma_bf16(tmem, ptx::sw128_kmajor_desc(qa + kb * 16384 + kk * 32),
+                         ptx::sw128_kmajor_desc(ka + kb * 8192 + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
+      ptx::umma_commit(&bars[2]);
+    } else {
+      atomicOr(a.status, RTV_DEV_TIMEOUT);
+    }
+  }
+  __syncwarp();   // the rest of warp 0 waits here, not spinning beside the issuing lane
+  // ---- softmax: a row (TMEM lane) per thread pair, 32 key columns each ----
+  const int r = 32 * quarter + lane;
+  const int s = r & 63;
+  const bool row_valid = s < a.S;
+  const int n_keys = suffix_tile ? a.S : min(64, a.P - 64 * rank);
+  // the Pi0 block mask hides the action tokens of the suffix from the state token (row s == 0)
+  const int n_vis = (a.mask_mode == RTV_MASK_PI0_BLOCK && suffix_tile && s == 0) ? 1 : n_keys;
+  if (!ptx::mbar_wait(&bars[2], 0, a.timeout_ns)) atomicOr(a.status, RTV_DEV_TIMEOUT);
+  ptx::tc_fence_after();
+  if (trace && tid == 0) trace[9] = ptx::globaltimer();
+  float x[32];
+  ptx::tmem_ld_32(tmem + lane_base + 32u * half, x);
+  if (trace && tid == 0) trace[10] = ptx::globaltimer();
+  float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    x[e] = 32 * half + e < n_vis ? x[e] * a.scale_log2 : -INFINITY;
+    m4[e & 3] = fmaxf(m4[e & 3], x[e]);
+  }
+  red_m[half][r] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+  __syncthreads();
+  const float mx = fmaxf(red_m[0][r], red_m[1][r]);
+  float l4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    x[e] = x[e] == -INFINITY ? 0.f : exp2f(x[e] - mx);
+    l4[e & 3] += x[e];
+  }
+  red_l[half][r] = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+  // P row: this thread's 32 keys = 4 chunks of 16 bytes, chunk-swizzled like a K-major operand tile
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    const int c = 4 * half + cc;
+    uint4 v;
+    v.x = ptx::pack_bf16x2(x[8 * cc], x[8 * cc + 1]);
+    v.y = ptx::pack_bf16x2(x[8 * cc + 2], x[8 * cc + 3]);
+    v.z = ptx::pack_bf16x2(x[8 * cc + 4], x[8 * cc + 5]);
+    v.w = ptx::pack_bf16x2(x[8 * cc + 6], x[8 * cc + 7]);
+    *reinterpret_cast<uint4*>(Ps + r * 128 + ((c ^ (r & 7)) << 4)) = v;
+  }
+  if (trace && tid == 0) trace[11] = ptx::globaltimer();
+  ptx::fence_proxy_async_smem();
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (trace && tid == 0) trace[3] = ptx::globaltimer();
+  const size_t part_base = (size_t)(g * HP + hp) * nch;   // slot of rank q: part_base + q
+  if (half == 0 && row_valid)
+    *reinterpret_cast<float2*>(a.part_ml + ((part_base + rank) * 128 + r) * 2) =
+        make_float2(mx, red_l[0][r] + red_l[1][r]);
+  if (tid == 0 && ok) {
+    ptx::tc_fence_after();
+    const uint32_t idesc = ptx::idesc_bf16_f32(128, D);
+    const uint32_t pa = ptx::smem_u32(Ps), va = ptx::smem_u32(Vs);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      ptx::umma_bf16(tmem, ptx::sw128_kmajor_desc(pa + kk * 32), ptx::sw128_kmajor_desc(va + kk * 32), idesc,
+                     kk != 0 ? 1u : 0u);
+    ptx::umma_commit(&bars[3]);
+  }
+  __syncwarp();
+  if (!ptx::mbar_wait(&bars[3], 0, a.timeout_ns)) atomicOr(a.status, RTV_DEV_TIMEOUT);
+  ptx::tc_fence_after();
+  if (trace && tid == 0) trace[4] = ptx::globaltimer();
+  // unnormalised O rows -> the Q tile's space (free since S was computed),
+  // chunk-swizzled; each thread of a pair takes half of the D columns
+#pragma unroll 1
+  for (int cb = 0; cb < D / 64; ++cb) {
+    const int col = (D / 2) * half + 32 * cb;
+    float v[32];
+    ptx::tmem_ld_32(tmem + lane_base + (uint32_t)col, v);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      uint4 u;
+      u.x = ptx::pack_bf16x2(v[8 * e], v[8 * e + 1]);
+      u.y = ptx::pack_bf16x2(v[8 * e + 2], v[8 * e + 3]);
+      u.z = ptx::pack_bf16x2(v[8 * e + 4], v[8 * e + 5]);
+      u.w = ptx::pack_bf16x2(v[8 * e + 6], v[8 * e + 7]);
+      const int c = col / 8 + e;   // 16-byte chunk of the row
+      *reinterpret_cast<uint4*>(Qs + r * (D * 2) + ((c ^ (r & 7)) << 4)) = u;
+    }
+  }
+  if (trace && tid == 0) trace[12] = ptx::globaltimer();
+  ptx::tc_fence_before();
+  __syncthreads();
+  // out to global memory, one coalesced row per warp step (valid rows only)
+  {
+    __nv_bfloat16* po = a.part_o + (part_base + rank) * 128 * D;
+    for (int rr = warp; rr < 128; rr += 8) {
+      if ((rr & 63) >= a.S) continue;
+      for (int c = lane; c < CPR; c += 32)
+        *reinterpret_cast<uint4*>(po + (size_t)rr * D + c * 8) =
+            *reinterpret_cast<const uint4*>(Qs + rr * (D * 2) + ((c ^ (rr & 7)) << 4));
+    }
+  }
+  if (trace && tid == 0) trace[5] = ptx::globaltimer();
+  // release / acquire at cluster scope: every rank's partials are visible
+  ptx::cluster_sync();
+  if (trace && tid == 0) trace[6] = trace[7] = ptx::globaltimer();
+  // combine: the pair's 2*S valid rows are split evenly over the ranks; a warp
+  // takes two of its rank's rows at a time and issues every load of both
+  // before reducing (ranks summed in order)
+  const int nvalid = 2 * a.S;
+  const int rpc = (nvalid + nch - 1) / nch;
+  const int v0 = rank * rpc, v1 = min(nvalid, v0 + rpc);
+  for (int vb = v0 + warp; vb < v1; vb += 16) {
+    int rows[2];
+    bool has[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int vi = vb + 8 * u;
+      has[u] = vi < v1;
+      const int hs = has[u] ? vi / a.S : 0;
+      rows[u] = has[u] ? hs * 64 + (vi - hs * a.S) : 0;
+    }
+    float mq[2] = {-INFINITY, -INFINITY}, lq[2] = {0.f, 0.f};
+    uint4 v[2][16];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (has[u] && lane < nch) {
+        const float2 ml =
+            __ldcg(reinterpret_cast<const float2*>(a.part_ml + ((part_base + lane) * 128 + rows[u]) * 2));
+        mq[u] = ml.x;
+        lq[u] = ml.y;
+      }
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        if (has[u] && q < nch && lane < CPR)
+          v[u][q] = __ldcg(reinterpret_cast<const uint4*>(a.part_o + ((part_base + q) * 128 + rows[u]) * D + lane * 8));
+    }
+    if (trace && tid == 0 && vb == v0) trace[13] = ptx::globaltimer();
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (!has[u]) continue;   // uniform across the warp
+      const float m_all = warp_max(mq[u]);
+      const float wq = (lane < nch && mq[u] != -INFINITY) ? exp2f(mq[u] - m_all) : 0.f;
+      const float inv = 1.f / warp_sum(wq * lq[u]);
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const float wqq = __shfl_sync(0xffffffffu, wq, q);
+        if (q < nch && lane < CPR) {
+          const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&v[u][q]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(v2[e]);
+            acc[2 * e] = fmaf(wqq, f.x, acc[2 * e]);
+            acc[2 * e + 1] = fmaf(wqq, f.y, acc[2 * e + 1]);
+          }
+        }
+      }
+      if (lane < CPR) {
+        uint4 out;
+        out.x = ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv);
+        out.y = ptx::pack_bf16x2(acc[2] * inv, acc[3] * inv);
+        out.z = ptx::pack_bf16x2(acc[4] * inv, acc[5] * inv);
+        out.w = ptx::pack_bf16x2(acc[6] * inv, acc[7] * inv);
+        const int j = 2 * hp + (rows[u] >> 6);
+        *reinterpret_cast<uint4*>(a.o + ts_offset(g * a.S + (rows[u] & 63), j * D + lane * 8, a.n_mma)) = out;
+      }
+      if (trace && tid == 0 && vb == v0) trace[14 + u] = ptx::globaltimer();
+    }
+  }
+  if (trace && tid == 0) trace[8] = ptx::globaltimer();
+  __syncthreads();
+  if (warp == 0) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, TCOLS);
+  }
+  // never leave with a copy still landing in this CTA's shared memory
+  if (tid == 0 && !ok) {
+    ptx::mbar_wait(&bars[0], 0, a.timeout_ns);
+    ptx::mbar_wait(&bars[1], 0, a.timeout_ns);
+  }
+}
+
+// Prefix tiles of the tensor-core attention, from the cached prefix
+// [L][2][Bmax][Hkv][Pmax][D]: keys [l][b][h][tile][64][D] and values
+// transposed [l][b][h][tile][D][64], both tiled and pre-swizzled.  One thread
+// per 8 consecutive features of one key.
+__global__ void prefix_tile_kernel(const __nv_bfloat16* __restrict__ kv, __nv_bfloat16* __restrict__ pkt,
+                                   __nv_bfloat16* __restrict__ pvt, int L, int B, int P, int Hkv, int D, int Bmax,
+                                   int Pmax, int ntile_max) {
+  const size_t n = (size_t)L * B * Hkv * P * (D / 8);
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const int d0 = 8 * (int)(i % (D / 8));
+    size_t rest = i / (D / 8);
+    const int key = (int)(rest % P);
+    rest /= P;
+    const int h = (int)(rest % Hkv);
+    rest /= Hkv;
+    const int b = (int)(rest % B);
+    const int l = (int)(rest / B);
+    const size_t src_k = ((((size_t)l * 2 + 0) * Bmax + b) * Hkv + h) * Pmax * D + (size_t)key * D + d0;
+    const size_t src_v = ((((size_t)l * 2 + 1) * Bmax + b) * Hkv + h) * Pmax * D + (size_t)key * D + d0;
+    const size_t tile = (((size_t)l * Bmax + b) * Hkv + h) * ntile_max + key / 64;
+    const int kr = key & 63;
+    *reinterpret_cast<uint4*>(pkt + tile * 64 * D + ts_offset(kr, d0, 64)) = *reinterpret_cast<const uint4*>(kv + src_k);
+    const uint4 vv = *reinterpret_cast<const uint4*>(kv + src_v);
+    const __nv_bfloat16* ve = reinterpret_cast<const __nv_bfloat16*>(&vv);
+    __nv_bfloat16* vt = pvt + tile * 64 * D;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) vt[ts_offset(d0 + e, kr, D)] = ve[e];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// ---------------------------------------------------------------------------
 // Step kernel: output head of the previous Euler step and suffix embedding
 // of the next ("DM0.5 reading guide", sec. 5.2 action_out_proj /
 // action_in_proj / state token, sec. 5.3 Euler update x <- x - dt * v).
@@ -895,8 +1248,15 @@ struct FastPath {
   __nv_bfloat16 *w_aiT = nullptr, *w_spT = nullptr;
   __nv_bfloat16 *qb = nullptr, *ksb = nullptr, *vsb = nullptr, *ob = nullptr, *mb = nullptr, *hb = nullptr;
   float* ssp = nullptr;
-  __nv_bfloat16* att_po = nullptr;   // attention partial rows [Gmax][Hq][16][64][D]
-  float* att_pml = nullptr;          // their (max, sum)       [Gmax][Hq][16][64][2]
+  // attention partial rows [Gmax][Hq][16][64][D] (the tensor-core kernel
+  // indexes the same storage as [Gmax][Hq/2][16][128][D]) and their (max, sum)
+  __nv_bfloat16* att_po = nullptr;
+  float* att_pml = nullptr;
+  // tensor-core attention (head pairs sharing a KV head): tiled operands
+  bool tc_attn = false;
+  int ntile_max = 0;                 // 64-key tiles of the longest prefix
+  __nv_bfloat16 *qt = nullptr, *kts = nullptr, *vts = nullptr;   // q of head pairs, suffix K and V^T tiles
+  __nv_bfloat16 *pkt = nullptr, *pvt = nullptr;                  // prefix K and V^T tiles, all layers
   int num_sms = 148;
   int max_cluster = 8;
   int gemm_fit_small[17] = {0};   // co-resident GEMM clusters by size, at the smem_cap budget (diagnostic)
@@ -1033,6 +1393,34 @@ cudaError_t launch_attn(const AttnArgs& a, int nchunk, int G, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
+template <int D>
+cudaError_t configure_attn_tc() {
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       attn_tc_smem_bytes(D));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
+}
+
+template <int D>
+cudaError_t launch_attn_tc(const AttnTcArgs& a, int nchunk, int G, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nchunk, a.Hq / 2, G);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = attn_tc_smem_bytes(D);
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeClusterDimension;
+  attrs[0].val.clusterDim.x = nchunk;
+  attrs[0].val.clusterDim.y = 1;
+  attrs[0].val.clusterDim.z = 1;
+  attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, attn_tc_kernel<D>, a);
+}
+
 cudaError_t launch_step(const StepArgs& a, int rows, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(rows, 1, 1);
@@ -1073,7 +1461,8 @@ rtv_status fast_create(rtv_ctx* ctx) {
   int dev = ctx->device;
   if (configure_gemm<GM_QKV>() != cudaSuccess || configure_gemm<GM_O>() != cudaSuccess ||
       configure_gemm<GM_GU>() != cudaSuccess || configure_gemm<GM_DOWN>() != cudaSuccess ||
-      configure_attn<128>() != cudaSuccess || configure_attn<256>() != cudaSuccess) {
+      configure_attn<128>() != cudaSuccess || configure_attn<256>() != cudaSuccess ||
+      configure_attn_tc<128>() != cudaSuccess || configure_attn_tc<256>() != cudaSuccess) {
     cudaGetLastError();
     return RTV_ERR_CUDA;
   }
@@ -1116,6 +1505,17 @@ rtv_status fast_create(rtv_ctx* ctx) {
             alloc((void**)&fp->att_pml, (size_t)ctx->Gmax * k.n_q_heads * 16 * 64 * 2 * 4) &&
             alloc((void**)&fp->ksb, (size_t)ctx->Gmax * ctx->KV * S * 2) &&
             alloc((void**)&fp->vsb, (size_t)ctx->Gmax * ctx->KV * S * 2);
+  // tensor-core attention: both heads of a pair must share their KV head
+  fp->tc_attn = k.n_q_heads % 2 == 0 && (k.n_q_heads / k.n_kv_heads) % 2 == 0;
+  fp->ntile_max = (k.max_prefix_len + 63) / 64;
+  if (ok && fp->tc_attn) {
+    const size_t D = k.head_dim, Hkv = k.n_kv_heads;
+    ok = alloc((void**)&fp->qt, (size_t)ctx->Gmax * (k.n_q_heads / 2) * 128 * D * 2) &&
+         alloc((void**)&fp->kts, (size_t)ctx->Gmax * Hkv * 64 * D * 2) &&
+         alloc((void**)&fp->vts, (size_t)ctx->Gmax * Hkv * 64 * D * 2) &&
+         alloc((void**)&fp->pkt, (size_t)k.n_layers * k.max_batch * Hkv * fp->ntile_max * 64 * D * 2) &&
+         alloc((void**)&fp->pvt, (size_t)k.n_layers * k.max_batch * Hkv * fp->ntile_max * 64 * D * 2);
+  }
   if (!ok) {
     for (void* p : fp->allocs) cudaFree(p);
     delete fp;
@@ -1148,8 +1548,8 @@ void fast_trace_report(rtv_ctx* ctx) {
   const char* nm[5] = {"qkv", "o", "gu", "down", "attention"};
   const char* ev[2][15] = {{"start", "w_issued", "pdl", "first_full", "mma_issued", "done", "copied", "recv", "end",
                            "prefetched", "arrived", "iter0", "exit", "part", "entry"},
-                          {"start", "pdl", "tile0", "loop_end", "merged", "entry", "pushed", "synced", "end", "", "", "",
-                           "", "", ""}};
+                          {"start", "pdl", "tile0", "loop_end", "merged", "entry", "pushed", "synced", "end", "s_seen",
+                           "s_loaded", "p_stored", "o_staged", "cmb_issued", "cmb_row0"}};
   unsigned long long t_ref = ~0ull;
   for (int i = 0; i < 5; ++i)
     for (int c = 0; c < fp->trace_ctas[i]; ++c)
@@ -1160,8 +1560,9 @@ void fast_trace_report(rtv_ctx* ctx) {
     fprintf(stderr, "[rtv trace] %s (%d CTAs), us after the first traced start: min / median / max\n", nm[i],
             fp->trace_ctas[i]);
     const int order_e[15] = {0, 1, 2, 3, 4, 5, 13, 14, 6, 9, 7, 10, 11, 8, 12};
+    const int order_a[15] = {0, 1, 2, 9, 10, 11, 3, 4, 12, 5, 6, 7, 13, 14, 8};
     for (int ei = 0; ei < 15; ++ei) {
-      const int e = order_e[ei];
+      const int e = i == 4 ? order_a[ei] : order_e[ei];
       if (!ev[i == 4][e][0]) continue;
       std::vector<double> v;
       for (int c = 0; c < fp->trace_ctas[i]; ++c) {
@@ -1190,6 +1591,21 @@ void fast_trace_report(rtv_ctx* ctx) {
 }
 
 bool fast_supports_prefix(rtv_ctx*, int) { return true; }
+
+rtv_status fast_prefix_update(rtv_ctx* ctx, int batch, int prefix_len, cudaStream_t st) {
+  FastPath* fp = ctx->fast;
+  if (!fp || !fp->tc_attn) return RTV_OK;
+  const rtv_expert_config& k = ctx->cfg;
+  prefix_tile_kernel<<<4 * fp->num_sms, 256, 0, st>>>((const __nv_bfloat16*)ctx->prefix_kv, fp->pkt, fp->pvt,
+                                                     k.n_layers, batch, prefix_len, k.n_kv_heads, k.head_dim,
+                                                     k.max_batch, k.max_prefix_len, fp->ntile_max);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    ctx->last_error = std::string("prefix tiling launch: ") + cudaGetErrorString(e);
+    return RTV_ERR_CUDA;
+  }
+  return RTV_OK;
+}
 
 rtv_status fast_load(rtv_ctx* ctx, const rtv_tensor*, int) {
   FastPath* fp = ctx->fast;
@@ -1353,6 +1769,37 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
   at.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
   const size_t kv_layer = (size_t)k.max_batch * k.n_kv_heads * k.max_prefix_len * D;
 
+  // tensor-core attention when the pair layout applies and every key tile has
+  // a rank (RTV_ATTN=mma selects the warp-MMA kernel instead)
+  const int ntp = (P + 63) / 64;
+  const char* attn_env = getenv("RTV_ATTN");
+  const bool tc_att = fp->tc_attn && ntp + 1 <= 16 && ntp <= fp->ntile_max &&
+                      !(attn_env && strcmp(attn_env, "mma") == 0);
+  AttnTcArgs atc{};
+  if (tc_att) {
+    base.qt = fp->qt;
+    base.kts = fp->kts;
+    base.vts = fp->vts;
+    atc.qt = fp->qt;
+    atc.kts = fp->kts;
+    atc.vts = fp->vts;
+    atc.o = fp->ob;
+    atc.part_o = fp->att_po;
+    atc.part_ml = fp->att_pml;
+    atc.status = ctx->status;
+    atc.timeout_ns = k.barrier_timeout_ns;
+    atc.S = S;
+    atc.P = P;
+    atc.Hq = k.n_q_heads;
+    atc.Hkv = k.n_kv_heads;
+    atc.pbs = prefix_batch_stride;
+    atc.mask_mode = k.suffix_mask;
+    atc.ntile_max = fp->ntile_max;
+    atc.n_mma = n_mma;
+    atc.scale_log2 = at.scale_log2;
+  }
+  const size_t ptile_layer = (size_t)k.max_batch * k.n_kv_heads * fp->ntile_max * 64 * D;
+
   const bool tracing = fp->trace_armed && fp->trace != nullptr;
   fp->trace_armed = false;
   if (tracing) {
@@ -1360,7 +1807,7 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     fp->trace_ctas[1] = p_o.n_tiles * p_o.cs;
     fp->trace_ctas[2] = p_gu.n_tiles * p_gu.cs;
     fp->trace_ctas[3] = p_dn.n_tiles * p_dn.cs;
-    fp->trace_ctas[4] = nchunk * k.n_q_heads * G;
+    fp->trace_ctas[4] = tc_att ? (ntp + 1) * (k.n_q_heads / 2) * G : nchunk * k.n_q_heads * G;
   }
   auto tr = [&](int l, int i) -> unsigned long long* {
     return (tracing && l == 0) ? fp->trace + (size_t)i * 512 * kTraceRow : nullptr;
@@ -1376,10 +1823,18 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     a.w_tile0 = l * nq / 128;
     cudaError_t e = launch_gemm<GM_QKV>(a, p_qkv, st);
 
-    at.trace = tr(l, 4);
-    at.pk = (const __nv_bfloat16*)ctx->prefix_kv + (size_t)(2 * l) * kv_layer;
-    at.pv = (const __nv_bfloat16*)ctx->prefix_kv + (size_t)(2 * l + 1) * kv_layer;
-    if (e == cudaSuccess) e = D == 256 ? launch_attn<256>(at, nchunk, G, st) : launch_attn<128>(at, nchunk, G, st);
+    if (tc_att) {
+      atc.trace = tr(l, 4);
+      atc.pkt = fp->pkt + (size_t)l * ptile_layer;
+      atc.pvt = fp->pvt + (size_t)l * ptile_layer;
+      if (e == cudaSuccess)
+        e = D == 256 ? launch_attn_tc<256>(atc, ntp + 1, G, st) : launch_attn_tc<128>(atc, ntp + 1, G, st);
+    } else {
+      at.trace = tr(l, 4);
+      at.pk = (const __nv_bfloat16*)ctx->prefix_kv + (size_t)(2 * l) * kv_layer;
+      at.pv = (const __nv_bfloat16*)ctx->prefix_kv + (size_t)(2 * l + 1) * kv_layer;
+      if (e == cudaSuccess) e = D == 256 ? launch_attn<256>(at, nchunk, G, st) : launch_attn<128>(at, nchunk, G, st);
+    }
 
     a = base;
     a.trace = tr(l, 1);

@@ -113,6 +113,7 @@ extern "C" rtv_status rtv_set_prefix_kv_static(rtv_ctx* ctx, const void* kv, int
       s = RTV_ERR_CUDA;
     }
   }
+  if (s == RTV_OK && ctx->use_fast) s = rtv::fast_prefix_update(ctx, batch, prefix_len, st);
   if (prev >= 0 && prev != ctx->device) cudaSetDevice(prev);
   if (s != RTV_OK) return s;
   ctx->prefix_len = prefix_len;

@@ -446,6 +446,10 @@ rtv_status rtv_set_prefix_kv(rtv_ctx* ctx, const void* kv, int prefix_len, int b
                                       prefix_len, k.n_kv_heads, k.head_dim, k.max_batch, k.max_prefix_len, st);
   CK(cudaGetLastError());
   if (tmp) CK(cudaFreeAsync(tmp, st));
+  if (ctx->use_fast) {
+    const rtv_status fs = fast_prefix_update(ctx, batch, prefix_len, st);
+    if (fs != RTV_OK) return fs;
+  }
   ctx->prefix_len = prefix_len;
   ctx->prefix_batch = batch;
   ctx->have_prefix = true;

@@ -70,6 +70,35 @@ def test_pi0_two_layer_bf16_denoise_matches_oracle(cuda_ok):
     assert bf16_tolerance_ok(got, ref), (rel_l2(got, ref), np.max(np.abs(got - ref)))
 
 
+@pytest.mark.parametrize("prefix_len", [37, 64, 960, 961])
+def test_pi0_bf16_prefix_tiling_edges(cuda_ok, prefix_len):
+    """Prefix lengths at the attention's 64-key tile edges: one partial tile,
+    one full tile, the most tiles the tensor-core attention takes (15 prefix
+    tiles + the suffix tile), and one key more (the warp-MMA attention)."""
+    cfg = get_config("pi0-bf16", n_layers=1, prefix_len=prefix_len)
+    got, ref, _ = run_denoise(cfg, n_steps=2)
+    assert bf16_tolerance_ok(got, ref), (rel_l2(got, ref), np.max(np.abs(got - ref)))
+
+
+@pytest.mark.parametrize("variant", [
+    {"suffix_mask": "pi0_block"}, {"n_kv_heads": 2}, {"n_kv_heads": 8}, {"rope_theta": 0.0},
+])
+def test_pi0_bf16_attention_variants(cuda_ok, variant):
+    """Mask, grouped and ungrouped KV heads (8 KV heads: no head pair shares
+    one, so the warp-MMA attention runs), no RoPE."""
+    cfg = get_config("pi0-bf16", n_layers=2, prefix_len=200, **variant)
+    got, ref, _ = run_denoise(cfg, n_steps=2)
+    assert bf16_tolerance_ok(got, ref), (rel_l2(got, ref), np.max(np.abs(got - ref)))
+
+
+def test_warp_mma_attention_matches_oracle(cuda_ok, monkeypatch):
+    """The warp-MMA attention kernel, selected explicitly, on the full prefix."""
+    monkeypatch.setenv("RTV_ATTN", "mma")
+    cfg = get_config("pi0-bf16", n_layers=2)
+    got, ref, _ = run_denoise(cfg, n_steps=3)
+    assert bf16_tolerance_ok(got, ref), (rel_l2(got, ref), np.max(np.abs(got - ref)))
+
+
 def test_pi0_full_bf16_denoise_matches_oracle(cuda_ok):
     """The full 18-layer, 816-prefix, 10-step chunk, compared element by element."""
     cfg = get_config("pi0-bf16")
