@@ -154,8 +154,17 @@ __device__ __forceinline__ void bulk_copy_to_rank(uint32_t dst_cluster, uint32_t
       : "memory");
 }
 
+// Warp roles of a GEMM CTA: warp 0 loads, warp 1 issues the MMAs, and
+// kEpiWarps warps run the epilogue -- two per TMEM lane quarter, splitting
+// the token columns -- so that its latency chains overlap.
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kGemmThreads = 64 + kEpiThreads;
+
+// (Two CTAs fit an SM by registers, so a grid a little larger than the SM
+// count still runs in one wave.)
 template <int MODE>
-__global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const GemmArgs a) {
+__global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ float rs_s[64];
   const int n_mma = a.n_mma;
@@ -203,7 +212,6 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const GemmArgs a) {
   }
   __syncthreads();
   cluster_arrive_relaxed();
-  ptx::pdl_launch_dependents();
 
   // Weights do not depend on the previous kernel: the first ring-full of
   // weight boxes is requested before anyone waits on that kernel.  Nothing
@@ -227,6 +235,11 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const GemmArgs a) {
   __syncthreads();   // TMEM address published
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Dependents may launch only once this CTA holds its tensor memory: every
+  // kernel here allocates before it lets the next one start, so an
+  // allocation can only ever wait for CTAs of earlier kernels, which never
+  // wait on later ones.
+  ptx::pdl_launch_dependents();
 
   // After a bounded wait gives up, a role stops issuing copies and MMAs (so no
   // barrier ever sees an extra arrival), records the timeout, and still
@@ -278,7 +291,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const GemmArgs a) {
       if (trace) trace[TR_MMA_ISSUED] = ptx::globaltimer();
     }
   } else {
-    // ---- epilogue warps 2..5 ----
+    // ---- epilogue warps 2..9 ----
     const int tid = threadIdx.x - 64;
     ptx::pdl_wait();   // this role reads and writes what earlier kernels produced
     if (tid == 0) ptx::mbar_expect_tx(rbar, (uint32_t)(cs * n_own * 512));
@@ -293,12 +306,12 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const GemmArgs a) {
     const bool rope = MODE == GM_QKV && hh < a.Hq + a.Hkv;
     const uint32_t in_a = ptx::smem_u32(in_s);
     if (MODE == GM_O || MODE == GM_DOWN) {
-      for (int c = tid; c < n_own * 32; c += 128) {
+      for (int c = tid; c < n_own * 32; c += kEpiThreads) {
         const int tl = c >> 5, ch = c & 31;
         ptx::cp_async_16(in_a + (uint32_t)(c * 16), a.h + (size_t)(t_own0 + tl) * a.w + nt * 128 + ch * 4);
       }
     } else if (rope) {
-      for (int c = tid; c < n_own * 32; c += 128) {
+      for (int c = tid; c < n_own * 32; c += kEpiThreads) {
         const int tl = c >> 5, ch = c & 31;   // chunks 0-15: cos, 16-31: sin (64 floats each)
         const int s = (t_own0 + tl) % a.S;
         const float* src = (ch < 16 ? a.rope_cs : a.rope_sn) + (size_t)s * hd + dq0 + (ch & 15) * 4;
@@ -321,10 +334,11 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const GemmArgs a) {
     if (!ptx::mbar_wait(done, 0, a.timeout_ns)) atomicOr(a.status, RTV_DEV_TIMEOUT);
     ptx::tc_fence_after();
     if (trace && tid == 0) trace[TR_DONE] = ptx::globaltimer();
-    // accumulator -> this CTA's partial tile [token][feature]
+    // accumulator -> this CTA's partial tile [token][feature]; the two warps
+    // of a lane quarter take alternate 32-column chunks
     const int quarter = warp & 3;
     const int f = quarter * 32 + lane;
-    for (int c = 0; c < n_mma; c += 32) {
+    for (int c = 32 * ((warp - 2) >> 2); c < n_mma; c += 64) {
       float v[32];
       if (c + 16 < n_mma) {
         ptx::tmem_ld_32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c, v);
@@ -338,22 +352,21 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const GemmArgs a) {
     }
     ptx::tc_fence_before();
     ptx::fence_proxy_async_smem();
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
     if (trace && tid == 0) trace[TR_PART] = ptx::globaltimer();
     cluster_wait();   // entry phase: every rank has started and initialised its barriers
     if (trace && tid == 0) trace[TR_ENTRY] = ptx::globaltimer();
-    if (tid == 0) {
+    if (tid < cs) {   // one lane per destination rank
+      const int r = tid;
       const uint32_t part_a = ptx::smem_u32(part), recv_a = ptx::smem_u32(recv), rbar_a = ptx::smem_u32(rbar);
-      for (int r = 0; r < cs; ++r) {
-        const int o0 = r * per, no = max(0, min(a.T, o0 + per) - o0);
-        if (no == 0) continue;
+      const int o0 = r * per, no = max(0, min(a.T, o0 + per) - o0);
+      if (no > 0)
         bulk_copy_to_rank(ptx::mapa(recv_a + (uint32_t)(rank * per * 512), (uint32_t)r),
                           part_a + (uint32_t)(o0 * 512), (uint32_t)(no * 512), ptx::mapa(rbar_a, (uint32_t)r));
-      }
-      if (trace) trace[TR_COPIED] = ptx::globaltimer();
+      if (trace && tid == 0) trace[TR_COPIED] = ptx::globaltimer();
     }
     ptx::cp_async_wait_all();
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
     if (trace && tid == 0) trace[TR_PREFETCHED] = ptx::globaltimer();
     if (!ptx::mbar_wait(rbar, 0, a.timeout_ns)) atomicOr(a.status, RTV_DEV_TIMEOUT);
     if (trace && tid == 0) trace[TR_RECV] = ptx::globaltimer();
@@ -366,7 +379,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const GemmArgs a) {
     // one warp per token; lane l takes features (2l, 2l+1) and (2l+64, 2l+65)
     const int ew = warp - 2;
 #pragma unroll 1
-    for (int tl = ew; tl < n_own; tl += 4) {
+    for (int tl = ew; tl < n_own; tl += kEpiWarps) {
       const int t = t_own0 + tl;
       float2 x1 = make_float2(0.f, 0.f), x2 = make_float2(0.f, 0.f);
       for (int qr = 0; qr < cs; ++qr) {
@@ -1309,7 +1322,7 @@ cudaError_t launch_gemm(const GemmArgs& a, const GemmPlan& pl, cudaStream_t st) 
   auto kern = gemm_tc_kernel<MODE>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.cs, pl.n_tiles, 1);
-  cfg.blockDim = dim3(192, 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = st;
   cudaLaunchAttribute attrs[2];
@@ -1473,7 +1486,7 @@ rtv_status fast_create(rtv_ctx* ctx) {
     for (int big = 0; big < 2; ++big) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(cs, 1, 1);
-      cfg.blockDim = dim3(192, 1, 1);
+      cfg.blockDim = dim3(kGemmThreads, 1, 1);
       cfg.dynamicSmemBytes = big ? kDynSmemMax : fp->smem_cap;
       cudaLaunchAttribute at;
       at.id = cudaLaunchAttributeClusterDimension;
