@@ -70,6 +70,8 @@ __host__ __device__ __forceinline__ size_t ts_offset(int t, int k, int block_row
 struct GemmArgs {
   const __nv_bfloat16* wt;    // packed weights of this projection, all layers [R/128][K/64][128][64]
   const __nv_bfloat16* act;   // bf16 input, tiled [K/64][n_mma][64]
+  const uint8_t* pf;          // weights of the next projection, brought into L2 while this one runs
+  unsigned long long pf_bytes;
   float* h;                   // fp32 residual stream [T][w] (O, DOWN add into it)
   __nv_bfloat16* hb;          // next norm's input bf16(h * (1 + g_next)), tiled [w/64][n_mma][64] (written by O, DOWN)
   float* ssp;                 // sums of squares of h per 128-feature tile [T][w/128]
@@ -226,6 +228,14 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
         ptx::bulk_load_hint(base + b * L.stage_bytes, wsrc + (size_t)b * 8192, 16384u, &full[b], pol);
       }
       if (trace) trace[TR_W_ISSUED] = ptx::globaltimer();
+    } else if (lane == 2 && a.pf) {
+      // this CTA's share of the next projection's weights, into L2 (a hint)
+      const unsigned long long n_cta = (unsigned long long)gridDim.x * gridDim.y;
+      const unsigned long long share = ((a.pf_bytes + n_cta - 1) / n_cta + 15) & ~15ull;
+      const unsigned long long lo = share * ((unsigned long long)blockIdx.y * gridDim.x + blockIdx.x);
+      const unsigned long long hi = lo + share < a.pf_bytes ? lo + share : a.pf_bytes;
+      for (unsigned long long off = lo; off < hi; off += 32768)
+        ptx::prefetch_l2_bulk(a.pf + off, (uint32_t)(hi - off < 32768 ? hi - off : 32768));
     }
   } else if (warp == 1) {
     ptx::tmem_alloc(tmem_slot, ncols);
@@ -245,23 +255,30 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
   // barrier ever sees an extra arrival), records the timeout, and still
   // reaches every cluster barrier.
   if (warp == 0) {
-    // ---- producer: activation boxes once the previous kernel is done; remaining weight boxes ----
+    // ---- producers: lane 0 streams the remaining weight boxes as stages free
+    // up; lane 1 the activation boxes once the previous kernel is done (two
+    // issuing threads keep more copies in flight per SM) ----
     if (lane == 0) {
+      for (int b = first; b < nbox; ++b) {
+        const int s = b % NS, u = b / NS;
+        if (!ptx::mbar_wait(&empty[s], (u - 1) & 1, a.timeout_ns)) {
+          atomicOr(a.status, RTV_DEV_TIMEOUT);
+          break;
+        }
+        ptx::mbar_expect_tx(&full[s], 16384u);
+        ptx::bulk_load_hint(base + s * L.stage_bytes, wsrc + (size_t)b * 8192, 16384u, &full[s], pol);
+      }
+    } else if (lane == 1) {
       ptx::pdl_wait();
       if (trace) trace[TR_PDL] = ptx::globaltimer();
       for (int b = 0; b < nbox; ++b) {
         const int s = b % NS, u = b / NS;
-        uint8_t* st = base + s * L.stage_bytes;
-        if (b >= first) {
-          if (!ptx::mbar_wait(&empty[s], (u - 1) & 1, a.timeout_ns)) {
-            atomicOr(a.status, RTV_DEV_TIMEOUT);
-            break;
-          }
-          ptx::mbar_expect_tx(&full[s], 16384u);
-          ptx::bulk_load_hint(st, wsrc + (size_t)b * 8192, 16384u, &full[s], pol);
+        if (b >= NS && !ptx::mbar_wait(&empty[s], (u - 1) & 1, a.timeout_ns)) {
+          atomicOr(a.status, RTV_DEV_TIMEOUT);
+          break;
         }
         ptx::mbar_expect_tx(&full[s], act_box_bytes);
-        ptx::bulk_load(st + 16384, asrc + (size_t)b * n_mma * 64, act_box_bytes, &full[s]);
+        ptx::bulk_load(base + s * L.stage_bytes + 16384, asrc + (size_t)b * n_mma * 64, act_box_bytes, &full[s]);
       }
     }
   } else if (warp == 1) {
@@ -1294,9 +1311,12 @@ constexpr int kDynSmemMax = kSmemOptin - 2048;   // every kernel here uses < 2 K
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 // Split of one projection over CTAs: 128-row weight tiles x K slices (one
-// cluster per tile, at most 8 CTAs).  The smallest cluster that puts at
-// least one CTA on every SM is taken; the ring depth is then the largest
-// that fits the shared-memory budget.
+// cluster per tile).  A CTA's MMAs run at a fixed rate of about one 64-wide
+// box per 0.4 us, whatever the token count, so the K slice per CTA sets the
+// time: the smallest cluster that puts at least one CTA on every SM is
+// taken (up to 16 CTAs).  The ring depth is then the largest that fits the
+// shared-memory budget; clusters of 16 keep to the two-CTAs-per-SM budget so
+// that all of them are resident at once.
 GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T) {
   GemmPlan best;
   best.n_tiles = N / 128;
@@ -1309,7 +1329,7 @@ GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T) {
   const int nbox = best.kslice / 64;
   int stages = nbox;
   // a grid of at most one CTA per SM may use the whole shared memory for its ring
-  const int cap = best.n_tiles * best.cs <= fp->num_sms ? kDynSmemMax : fp->smem_cap;
+  const int cap = best.n_tiles * best.cs <= fp->num_sms && best.cs < 16 ? kDynSmemMax : fp->smem_cap;
   while (stages > 1 && gemm_smem_layout(stages, n_mma, best.cs, T).total > cap) --stages;
   best.stages = stages;
   best.smem = gemm_smem_layout(stages, n_mma, best.cs, T).total;
@@ -1501,7 +1521,7 @@ rtv_status fast_create(rtv_ctx* ctx) {
       (big ? fp->gemm_fit_large : fp->gemm_fit_small)[cs] = n;
     }
   }
-  fp->max_cluster = 8;
+  fp->max_cluster = 16;
   for (int c : {2, 4, 6, 8, 12, 16})
     fp->attn_fit[c] = k.head_dim == 256 ? attn_clusters_that_fit<256>(c, S) : attn_clusters_that_fit<128>(c, S);
   const size_t T = ctx->Tmax;
@@ -1834,6 +1854,8 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     a.act = fp->hb;
     a.K = w;
     a.w_tile0 = l * nq / 128;
+    a.pf = (const uint8_t*)(fp->w_o + (size_t)l * w * Q);
+    a.pf_bytes = (unsigned long long)w * Q * 2;
     cudaError_t e = launch_gemm<GM_QKV>(a, p_qkv, st);
 
     if (tc_att) {
@@ -1855,6 +1877,8 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     a.act = fp->ob;
     a.K = Q;
     a.w_tile0 = l * w / 128;
+    a.pf = (const uint8_t*)(fp->w_gu + (size_t)l * 2 * F * w);
+    a.pf_bytes = (unsigned long long)2 * F * w * 2;
     a.g_next = Lw.g_mlp;
     if (e == cudaSuccess) e = launch_gemm<GM_O>(a, p_o, st);
 
@@ -1864,6 +1888,8 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     a.act = fp->hb;
     a.K = w;
     a.w_tile0 = l * 2 * F / 128;
+    a.pf = (const uint8_t*)(fp->w_down + (size_t)l * w * F);
+    a.pf_bytes = (unsigned long long)w * F * 2;
     if (e == cudaSuccess) e = launch_gemm<GM_GU>(a, p_gu, st);
 
     a = base;
@@ -1872,6 +1898,8 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     a.act = fp->mb;
     a.K = F;
     a.w_tile0 = l * w / 128;
+    a.pf = (const uint8_t*)(fp->w_qkv + (size_t)((l + 1) % k.n_layers) * nq * w);
+    a.pf_bytes = (unsigned long long)nq * w * 2;
     a.g_next = (l + 1 < k.n_layers) ? ctx->W.layers[l + 1].g_attn : nullptr;
     if (e == cudaSuccess) e = launch_gemm<GM_DOWN>(a, p_dn, st);
     if (e != cudaSuccess) {
