@@ -48,6 +48,9 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="pi0-bf16")
     ap.add_argument("--n-steps", type=int, default=10, help="Euler steps per chunk")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="override the workload's layer count (profiling runs on smaller captures only; "
+                         "the JSON line then names the reduced depth)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds of the oracle sample")
     ap.add_argument("--trace", action="store_true",
@@ -225,11 +228,14 @@ def run_ours(args, info):
 
     from flow_matching_action_dm0_b200 import ActionExpert
     from flow_matching_action_dm0_b200 import replicas as R
-    from synthetic import f32_to_bf16_bits, get_config, make_noise, make_prefix_kv, make_state, make_weights
+    from synthetic import (f32_to_bf16_bits, get_config, make_draft, make_noise, make_prefix_kv, make_state,
+                           make_weights)
 
     dev = info.local_rank
     torch.cuda.set_device(dev)
     cfg = get_config(args.workload, n_steps=args.n_steps)
+    if args.layers > 0:
+        cfg = cfg.with_(n_layers=args.layers)
     weights = make_weights(cfg)
     kv = make_prefix_kv(cfg)
     noise = make_noise(cfg)
@@ -293,6 +299,23 @@ def run_ours(args, info):
     R.barrier(info, dev)
     e2e_ms = R.max_over_ranks(e0.elapsed_time(e1) / K, info, dev)
 
+    # FLASH verification of one draft chunk at the workload's taus: one expert
+    # evaluation of len(taus) suffixes plus the decision, host buffers in and
+    # out (the call waits for its result); device time per call, median
+    draft = make_draft(cfg)
+    taus = tuple(cfg.taus)
+    for _ in range(3):
+        ex.verify(draft, noise, state, taus, 0.05, cfg.gripper, want_dist=False, stream=stream)
+    v_ms = []
+    for _ in range(max(5, min(K, 20))):
+        v0, v1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        v0.record(stream)
+        ex.verify(draft, noise, state, taus, 0.05, cfg.gripper, want_dist=False, stream=stream)
+        v1.record(stream)
+        torch.cuda.synchronize(dev)
+        v_ms.append(v0.elapsed_time(v1))
+    verify_us = float(np.median(v_ms)) * 1000.0
+
     launches_per_call = ex.kernels_per_call(n)
     path = ex.path
     ex.close()
@@ -317,7 +340,8 @@ def run_ours(args, info):
         "vs_baseline": None,
         "dtype": cfg.dtype,
         "data": "synthetic",
-        "config": {"workload": args.workload, "n_steps": n, "batch": cfg.batch, "prefix_len": cfg.prefix_len,
+        "config": {"workload": args.workload if args.layers <= 0 else f"{args.workload} ({cfg.n_layers} layers)",
+                   "n_steps": n, "batch": cfg.batch, "prefix_len": cfg.prefix_len,
                    "layers": cfg.n_layers, "width": cfg.width, "parallelism": f"replicas x{info.world}",
                    "l2": "inputs larger than L2: 623 MB of weights stream from HBM every Euler step; no flush",
                    "path": path},
@@ -330,6 +354,10 @@ def run_ours(args, info):
                 "h2d_bytes_per_step": int(noise.nbytes + state.nbytes), "d2h_bytes_per_step": int(noise.nbytes)},
         "clocks": clk.summary(),
         "gpu_launches": int(launches_per_call * K) if launches_per_call > 0 else None,
+        "verify": {"taus": list(taus), "us_per_call": verify_us,
+                   "ratio_to_one_euler_step": verify_us / (ms * 1000.0 / n),
+                   "note": "one FLASH verification (len(taus) suffixes in one expert evaluation + decision), "
+                           "host buffers, device time per call (median)"},
     }
     if info.world == 1 and not args.no_cpu_baseline:
         per_step_s, k = oracle_step_seconds(cfg, args.cpu_seconds)

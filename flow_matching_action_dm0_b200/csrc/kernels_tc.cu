@@ -110,17 +110,17 @@ struct GemmSmem {
 // the receive buffer [cs * per][128] of the cluster reduction; the
 // epilogue's per-token inputs [per][128] (residual rows or RoPE cos/sin);
 // mbarriers.
-__host__ __device__ inline GemmSmem gemm_smem_layout(int stages, int n_mma, int cs, int T) {
+__host__ __device__ inline GemmSmem gemm_smem_layout(int stages, int n_mma, int cs, int T, bool with_in = true) {
   GemmSmem s;
   const int per = (T + cs - 1) / cs;
   s.stages = stages;
   s.stage_bytes = 16384 + n_mma * 128;
   s.ring_bytes = stages * s.stage_bytes;
   const int part_bytes = n_mma * 512;
-  s.part_off = part_bytes <= s.ring_bytes ? 0 : s.ring_bytes;
-  s.recv_off = s.ring_bytes > s.part_off + part_bytes ? s.ring_bytes : s.part_off + part_bytes;
+  s.part_off = 0;   // the partial tile overlays the ring: every MMA has completed when it is written
+  s.recv_off = s.ring_bytes > part_bytes ? s.ring_bytes : part_bytes;
   s.in_off = s.recv_off + cs * per * 512;   // [per][128] fp32 epilogue inputs of the owned tokens
-  s.bar_off = s.in_off + per * 512;
+  s.bar_off = s.in_off + (with_in ? per * 512 : 0);   // GU reads no per-token epilogue inputs
   s.total = s.bar_off + (2 * stages + 2) * 8 + 16 + 1024;   // barriers, TMEM slot, alignment slack
   return s;
 }
@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
   __shared__ float rs_s[64];
   const int n_mma = a.n_mma;
   const int cs = gridDim.x;
-  const GemmSmem L = gemm_smem_layout(a.stages, n_mma, cs, a.T);
+  const GemmSmem L = gemm_smem_layout(a.stages, n_mma, cs, a.T, MODE != GM_GU);
   // every CTA of the grid sees the same values, so a refusal is uniform across each cluster
   if (dynamic_smem_size() < (uint32_t)L.total || a.kslice < 64 || (a.kslice & 63) || a.stages < 1 || n_mma > 256 ||
       (n_mma & 15) || a.T > n_mma || cs > 16 || (a.T + cs - 1) / cs > 64) {
@@ -1311,29 +1311,47 @@ constexpr int kDynSmemMax = kSmemOptin - 2048;   // every kernel here uses < 2 K
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 // Split of one projection over CTAs: 128-row weight tiles x K slices (one
-// cluster per tile).  A CTA's MMAs run at a fixed rate of about one 64-wide
-// box per 0.4 us, whatever the token count, so the K slice per CTA sets the
-// time: the smallest cluster that puts at least one CTA on every SM is
-// taken (up to 16 CTAs).  The ring depth is then the largest that fits the
-// shared-memory budget; clusters of 16 keep to the two-CTAs-per-SM budget so
-// that all of them are resident at once.
-GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T) {
+// cluster per tile, up to 16 CTAs).  A CTA's MMAs run at a fixed rate of
+// about one 64-wide box per 0.4 us whatever the token count, and a wave of
+// CTAs costs a few microseconds of fixed latency (loads, exchange, epilogue),
+// so the split minimises waves x (fixed + boxes per CTA).  Two CTAs share an
+// SM when the ring fits the smem_cap budget (the ring is then the deepest
+// that does), otherwise one (the ring the deepest that fits the whole shared
+// memory); a cluster size is only usable as far as its clusters fit.  Ties
+// go to the smaller cluster (less reduction traffic).
+GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T, bool with_in) {
   GemmPlan best;
   best.n_tiles = N / 128;
+  double best_cost = 1e30;
+  constexpr double kFixedBoxes = 8.0;   // a wave's fixed latency, in MMA boxes (~3 us)
   for (int cs = 1; cs <= fp->max_cluster; cs <<= 1) {
     if (K % (cs * 64)) break;
-    best.cs = cs;
-    best.kslice = K / cs;
-    if (best.n_tiles * cs >= fp->num_sms) break;
+    if ((T + cs - 1) / cs > 64) continue;
+    const int nbox = K / cs / 64;
+    auto total = [&](int st) { return gemm_smem_layout(st, n_mma, cs, T, with_in).total; };
+    int stages = nbox;
+    while (stages > 1 && total(stages) > fp->smem_cap) --stages;
+    int per_sm = 2;
+    if (total(stages) > fp->smem_cap) {
+      per_sm = 1;
+      stages = nbox;
+      while (stages > 1 && total(stages) > kDynSmemMax) --stages;
+      if (total(stages) > kDynSmemMax) continue;
+    }
+    const int ctas = best.n_tiles * cs;
+    const int fit = per_sm * std::max(1, fp->gemm_fit_large[cs]);   // clusters resident at once
+    const int waves = std::max((ctas + per_sm * fp->num_sms - 1) / (per_sm * fp->num_sms),
+                               (best.n_tiles + fit - 1) / fit);
+    const double cost = waves * (kFixedBoxes + nbox);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best.cs = cs;
+      best.kslice = K / cs;
+      best.stages = stages;
+      best.smem = total(stages);
+    }
   }
-  const int nbox = best.kslice / 64;
-  int stages = nbox;
-  // a grid of at most one CTA per SM may use the whole shared memory for its ring
-  const int cap = best.n_tiles * best.cs <= fp->num_sms && best.cs < 16 ? kDynSmemMax : fp->smem_cap;
-  while (stages > 1 && gemm_smem_layout(stages, n_mma, best.cs, T).total > cap) --stages;
-  best.stages = stages;
-  best.smem = gemm_smem_layout(stages, n_mma, best.cs, T).total;
-  best.valid = best.kslice >= 64 && best.smem <= kDynSmemMax && (T + best.cs - 1) / best.cs <= 64;
+  best.valid = best.kslice >= 64 && best.smem > 0 && best.smem <= kDynSmemMax && (T + best.cs - 1) / best.cs <= 64;
   return best;
 }
 
@@ -1735,10 +1753,10 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
   const int S = ctx->S, T = G * S, w = k.width, F = k.mlp_dim, D = k.head_dim, Q = ctx->Q, KV = ctx->KV;
   const int n_mma = round_up(T, 16);
   const int nq = Q + 2 * KV;
-  const GemmPlan p_qkv = plan_gemm(fp, nq, w, n_mma, T);
-  const GemmPlan p_o = plan_gemm(fp, w, Q, n_mma, T);
-  const GemmPlan p_gu = plan_gemm(fp, 2 * F, w, n_mma, T);
-  const GemmPlan p_dn = plan_gemm(fp, w, F, n_mma, T);
+  const GemmPlan p_qkv = plan_gemm(fp, nq, w, n_mma, T, true);
+  const GemmPlan p_o = plan_gemm(fp, w, Q, n_mma, T, true);
+  const GemmPlan p_gu = plan_gemm(fp, 2 * F, w, n_mma, T, false);
+  const GemmPlan p_dn = plan_gemm(fp, w, F, n_mma, T, true);
   const int nk = P + S;
   const int nchunk = attn_chunks(fp, nk, k.n_q_heads * G);
   if (!(p_qkv.valid && p_o.valid && p_gu.valid && p_dn.valid) ||

@@ -507,6 +507,7 @@ rtv_status rtv_verify(rtv_ctx* ctx, const float* draft, const float* noise, cons
   CK(cudaMemcpyAsync(accepted_len, ctx->accepted, sizeof(int), cudaMemcpyDefault, st));
   CK(cudaMemcpyAsync(flags, ctx->flags, sizeof(unsigned), cudaMemcpyDefault, st));
   if (dist) CK(cudaMemcpyAsync(dist, ctx->dist, (size_t)n_taus * ctx->H * sizeof(float), cudaMemcpyDefault, st));
+  if (ctx->use_fast && getenv("RTV_TRACE")) fast_trace_report(ctx);
   return RTV_OK;
 }
 
