@@ -168,13 +168,14 @@ constexpr int kGemmThreads = 64 + kEpiThreads;
 template <int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ float rs_s[64];
+  constexpr int kMaxOwn = 160;   // tokens one rank reduces and finishes
+  __shared__ float rs_s[kMaxOwn];
   const int n_mma = a.n_mma;
   const int cs = gridDim.x;
   const GemmSmem L = gemm_smem_layout(a.stages, n_mma, cs, a.T, MODE != GM_GU);
   // every CTA of the grid sees the same values, so a refusal is uniform across each cluster
   if (dynamic_smem_size() < (uint32_t)L.total || a.kslice < 64 || (a.kslice & 63) || a.stages < 1 || n_mma > 256 ||
-      (n_mma & 15) || a.T > n_mma || cs > 16 || (a.T + cs - 1) / cs > 64) {
+      (n_mma & 15) || a.T > n_mma || cs > 16 || (a.T + cs - 1) / cs > kMaxOwn) {
     if (threadIdx.x == 0) atomicOr(a.status, RTV_DEV_BOUNDS);
     return;
   }
@@ -1326,7 +1327,7 @@ GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T, bool with
   constexpr double kFixedBoxes = 8.0;   // a wave's fixed latency, in MMA boxes (~3 us)
   for (int cs = 1; cs <= fp->max_cluster; cs <<= 1) {
     if (K % (cs * 64)) break;
-    if ((T + cs - 1) / cs > 64) continue;
+    if ((T + cs - 1) / cs > 160) continue;   // tokens per rank (kMaxOwn in the kernel)
     const int nbox = K / cs / 64;
     auto total = [&](int st) { return gemm_smem_layout(st, n_mma, cs, T, with_in).total; };
     int stages = nbox;
@@ -1351,7 +1352,7 @@ GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T, bool with
       best.smem = total(stages);
     }
   }
-  best.valid = best.kslice >= 64 && best.smem > 0 && best.smem <= kDynSmemMax && (T + best.cs - 1) / best.cs <= 64;
+  best.valid = best.kslice >= 64 && best.smem > 0 && best.smem <= kDynSmemMax && (T + best.cs - 1) / best.cs <= 160;
   return best;
 }
 
