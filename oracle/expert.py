@@ -46,6 +46,10 @@ Where the pages are silent the plainest reading is taken:
   R6 GELU tanh approximation in the gated MLP.
   R7 biases only on state_proj, action_in/out_proj and the time MLP.
   R8 only the H action rows produce velocity; the state row is discarded.
+  R10 FP8 MLP (BASELINE's FP8 configuration): gate/up/down given as E4M3
+     codes with one fp32 scale per output row; W = decode(code) * scale,
+     everything else unchanged (bf16 activations, fp32 accumulation on the
+     device; fp64 here).
   R9 verify: per-row L2 distance over all action dims, strict d < delta,
      accepted length = longest prefix passing at every tau, one eps shared by
      all taus, gripper switch = sign (value > 0) change between consecutive
@@ -69,9 +73,35 @@ FLAG_SWITCH = 2           # gripper switch inside the draft chunk  [FLASH] 03.3
 FLAG_SWITCH_IN_PREFIX = 4  # a switch lies inside the accepted prefix
 
 
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """Values of FP8 E4M3 codes ([DM0.5] sec. 6.3 names FP8 E4M3 for the MLP
+    projections): bit 7 the sign, bits 6-3 the exponent with bias 7, bits 2-0
+    the mantissa; exponent 0 holds the subnormals (m/8) * 2^-6, every other
+    exponent (1 + m/8) * 2^(e-7); the code S.1111.111 is NaN and there are no
+    infinities (largest finite value 448)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c >> 7, -1.0, 1.0)
+    e = (c >> 3) & 15
+    m = c & 7
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2((e - 7).astype(F64)))
+    return np.where((e == 15) & (m == 7), np.nan, sign * mag)
+
+
 def to_f64(weights: Dict[str, np.ndarray]) -> Dict[str, np.ndarray]:
-    """fp64 copies of the given parameters (their values are unchanged)."""
-    return {k: np.asarray(v, dtype=F64) for k, v in weights.items()}
+    """fp64 values of the given parameters.  A matrix given as FP8 E4M3 codes
+    (uint8) is decoded and multiplied row by row by its fp32 scale (the
+    tensor of the same name ending in ".s"): BASELINE's FP8 MLP storage,
+    one scale per output channel."""
+    out: Dict[str, np.ndarray] = {}
+    for k, v in weights.items():
+        if k.endswith(".s"):
+            continue
+        a = np.asarray(v)
+        if a.dtype == np.uint8:
+            out[k] = e4m3_decode(a) * np.asarray(weights[k[:-2] + ".s"], dtype=F64)[:, None]
+        else:
+            out[k] = a.astype(F64)
+    return out
 
 
 # ---------------------------------------------------------------------------

@@ -1,8 +1,8 @@
 """Seeded synthetic inputs shared by the oracle and the CUDA path.
 
 This module only draws random numbers and lays them out: workload shapes,
-per-tensor seeded normal draws, and the bf16 storage rounding of inputs that
-are *given* in bf16.  It holds none of the method's arithmetic (no norm, no
+per-tensor seeded normal draws, and the bf16 / FP8 E4M3 storage encoding of
+inputs that are *given* in those formats.  It holds none of the method's arithmetic (no norm, no
 attention, no time embedding, no Euler step), so the oracle and the CUDA
 path can both use it without sharing any computation.
 """
@@ -10,6 +10,7 @@ path can both use it without sharing any computation.
 from .configs import CONFIGS, ExpertShape, get_config  # noqa: F401
 from .gen import (  # noqa: F401
     bf16_bits_to_f32,
+    e4m3_encode,
     f32_to_bf16_bits,
     make_draft,
     make_noise,

@@ -15,6 +15,12 @@ camera/robot data, which are not available):
 
 bf16 inputs are produced by round-to-nearest-even of the float32 draw; both
 the oracle and the CUDA path receive the same rounded values.
+
+In an FP8-MLP workload the gate/up/down matrices are *given* in FP8 E4M3
+storage with one fp32 scale per output row (BASELINE's FP8 configuration):
+the float32 draw of a row is divided by scale = max|row| / 448 and rounded to
+the nearest E4M3 value (ties to even).  The codes and scales are the inputs;
+what an E4M3 code means is decoded by each side on its own.
 """
 
 from __future__ import annotations
@@ -60,6 +66,27 @@ def round_to_bf16(a: np.ndarray) -> np.ndarray:
     return bf16_bits_to_f32(f32_to_bf16_bits(a))
 
 
+E4M3_MAX = 448.0
+
+
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    """E4M3 codes (uint8: sign, 4 exponent bits with bias 7, 3 mantissa bits;
+    no infinities) of float32 values with |x| <= 448, rounded to the nearest
+    representable value, ties to even (storage encoding of given inputs)."""
+    x = np.asarray(x, dtype=np.float32)
+    a = np.abs(x).astype(np.float64)
+    # quantum of the binade holding a: 2^(e-3) for normals (e >= -6), 2^-9 below 2^-6
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -6)))
+    q = 2.0 ** (e - 3)
+    v = np.minimum(np.rint(a / q) * q, E4M3_MAX)          # numpy rint: half to even
+    sub = v < 2.0 ** -6
+    ev = np.floor(np.log2(np.where(sub, 1.0, v)))           # exponent of the rounded value
+    mant = np.where(sub, np.rint(v / 2.0 ** -9), np.rint((v / 2.0 ** ev - 1.0) * 8.0))
+    expf = np.where(sub, 0, ev + 7)
+    code = (np.signbit(x).astype(np.uint32) << 7) | (expf.astype(np.uint32) << 3) | mant.astype(np.uint32)
+    return code.astype(np.uint8)
+
+
 # ---------------------------------------------------------------------------
 # weights
 # ---------------------------------------------------------------------------
@@ -86,6 +113,8 @@ def weight_names(cfg: ExpertShape) -> List[Tuple[str, Tuple[int, ...]]]:
             (p + "up_proj.w", (f, w)),
             (p + "down_proj.w", (w, f)),
         ]
+        if cfg.mlp_dtype == "fp8_e4m3":
+            out += [(p + "gate_proj.s", (f,)), (p + "up_proj.s", (f,)), (p + "down_proj.s", (w,))]
     out += [("final_norm.g", (w,)), ("action_out_proj.w", (a, w)), ("action_out_proj.b", (a,))]
     return out
 
@@ -95,11 +124,22 @@ def make_weights(cfg: ExpertShape, seed: int | None = None) -> Dict[str, np.ndar
 
     In a "bf16" workload every 2-D matrix holds bf16-representable values
     (it is stored and streamed as bf16); 1-D biases and gains stay float32.
+    In an FP8-MLP workload gate/up/down are uint8 E4M3 codes, each with a
+    float32 per-row scale under the name ending in ".s".
     """
     seed = cfg.seed if seed is None else seed
+    fp8 = cfg.mlp_dtype == "fp8_e4m3"
     ws: Dict[str, np.ndarray] = {}
     for name, shape in weight_names(cfg):
+        if fp8 and name.endswith("_proj.s"):
+            continue   # written with its matrix below
         a = _normal(seed, name, shape, cfg.weight_std)
+        if fp8 and name.split(".")[-2] in ("gate_proj", "up_proj", "down_proj"):
+            amax = np.max(np.abs(a), axis=1)
+            scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+            ws[name] = e4m3_encode(a / scale[:, None])
+            ws[name[:-2] + ".s"] = scale
+            continue
         if cfg.dtype == "bf16" and len(shape) == 2:
             a = round_to_bf16(a)
         ws[name] = a

@@ -357,3 +357,48 @@ def test_batch_elements_are_independent():
     both = O.denoise(W, cfg, noise, state, kv, 3)
     one = O.denoise(W, cfg, noise[1:], state[1:], kv[:, :, 1:], 3)
     np.testing.assert_array_equal(both[1], one[0])
+
+
+# ---------------------------------------------------------------------------
+# FP8 E4M3 MLP weights
+# ---------------------------------------------------------------------------
+
+def test_e4m3_decode_fixed_codes():
+    """Codes whose values the format fixes: zero, one, the extremes of both
+    ranges, a subnormal, halves, and NaN."""
+    codes = {0x00: 0.0, 0x38: 1.0, 0x30: 0.5, 0x3C: 1.5, 0x40: 2.0, 0x7E: 448.0, 0xFE: -448.0,
+             0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0xB8: -1.0, 0x77: 240.0}
+    got = O.e4m3_decode(np.array(list(codes), dtype=np.uint8))
+    assert np.array_equal(got, np.array(list(codes.values())))
+    assert np.isnan(O.e4m3_decode(np.array([0x7F, 0xFF], dtype=np.uint8))).all()
+    assert np.signbit(O.e4m3_decode(np.array([0x80], dtype=np.uint8)))[0]
+
+
+def test_e4m3_decode_matches_torch_float8_for_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = O.e4m3_decode(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+
+
+def test_fp8_mlp_weights_within_the_format_bound():
+    """Decoded FP8 weights (decode x per-row scale) stay within E4M3's rounding
+    bound of the draw they encode: relative 2^-4 for normal values, absolute
+    scale * 2^-10 for subnormal ones; each row's largest magnitude is exact."""
+    from synthetic.gen import _normal
+    cfg = get_config("pi0-fp8mlp", n_layers=1, width=256, mlp_dim=512, n_q_heads=2, head_dim=128)
+    raw = make_weights(cfg)
+    W = O.to_f64(raw)
+    for name in ("gate_proj", "up_proj", "down_proj"):
+        key = f"layers.0.{name}.w"
+        draw = _normal(cfg.seed, key, raw[key].shape, cfg.weight_std).astype(np.float64)
+        scale = raw[f"layers.0.{name}.s"].astype(np.float64)[:, None]
+        err = np.abs(W[key] - draw)
+        normal = np.abs(draw) / scale >= 2.0 ** -6
+        assert np.all(err[normal] <= 2.0 ** -4 * np.abs(draw)[normal] * (1 + 1e-6))
+        assert np.all(err[~normal] <= (scale * 2.0 ** -10 * (1 + 1e-6) + 0 * err)[~normal])
+        rows = np.arange(draw.shape[0])
+        amax_idx = np.argmax(np.abs(draw), axis=1)
+        assert np.allclose(W[key][rows, amax_idx], draw[rows, amax_idx], rtol=1e-6, atol=0)
