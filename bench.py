@@ -48,6 +48,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="pi0-bf16")
     ap.add_argument("--n-steps", type=int, default=10, help="Euler steps per chunk")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="independent chunks per call, each with its own prefix (default: the workload's)")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the workload's layer count (profiling runs on smaller captures only; "
                          "the JSON line then names the reduced depth)")
@@ -236,6 +238,8 @@ def run_ours(args, info):
     cfg = get_config(args.workload, n_steps=args.n_steps)
     if args.layers > 0:
         cfg = cfg.with_(n_layers=args.layers)
+    if args.batch > 0:
+        cfg = cfg.with_(batch=args.batch)
     weights = make_weights(cfg)
     kv = make_prefix_kv(cfg)
     noise = make_noise(cfg)
@@ -323,7 +327,7 @@ def run_ours(args, info):
     if not info.is_main:
         return
     peaks, peak_kind = load_peaks()
-    bytes_step = algorithmic_bytes_per_step(cfg)
+    bytes_step = algorithmic_bytes_per_step(cfg, batch=cfg.batch)
     bytes_chunk = bytes_step * n
     achieved = bytes_chunk / (ms * 1e-3) / 1e9
     peak = float(peaks["hbm_gbs"])
@@ -345,7 +349,7 @@ def run_ours(args, info):
                    "layers": cfg.n_layers, "width": cfg.width, "parallelism": f"replicas x{info.world}",
                    "l2": "inputs larger than L2: 623 MB of weights stream from HBM every Euler step; no flush",
                    "path": path},
-        "chunks_per_s": info.world * 1000.0 / ms,
+        "chunks_per_s": info.world * cfg.batch * 1000.0 / ms,
         "roofline": {"bound": "hbm", "kernel": "whole denoise graph (all kernels of one chunk)",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_kind": f"{peak_kind} hbm_gbs", "algorithmic_bytes_per_launch": bytes_chunk,

@@ -67,9 +67,28 @@ __host__ __device__ __forceinline__ size_t ts_offset(int t, int k, int block_row
   return ((size_t)(k >> 6) * block_rows + t) * 64 + ((((k >> 3) & 7) ^ (t & 7)) << 3) + (k & 7);
 }
 
+// Two E4M3 codes (low byte first) -> two bf16 values, exactly: the hardware
+// conversion to f16 holds every E4M3 value, and so does bf16.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two) {
+  uint32_t h2;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h2) : "r"(two));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+  return ptx::pack_bf16x2(f.x, f.y);
+}
+__device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 v) {
+  uint4 r;
+  r.x = e4m3x2_to_bf16x2(v.x & 0xFFFFu);
+  r.y = e4m3x2_to_bf16x2(v.x >> 16);
+  r.z = e4m3x2_to_bf16x2(v.y & 0xFFFFu);
+  r.w = e4m3x2_to_bf16x2(v.y >> 16);
+  return r;
+}
+
 struct GemmArgs {
   const __nv_bfloat16* wt;    // packed weights of this projection, all layers [R/128][K/64][128][64]
   const __nv_bfloat16* act;   // bf16 input, tiled [K/64][n_mma][64]
+  const uint8_t* wt8;         // FP8 E4M3 weights [R/128][K/64][128][64] bytes (GU, DOWN of an FP8 MLP), or nullptr
+  const float* wscale;        // their per-row scales in packed row order, this layer
   const uint8_t* pf;          // weights of the next projection, brought into L2 while this one runs
   unsigned long long pf_bytes;
   float* h;                   // fp32 residual stream [T][w] (O, DOWN add into it)
@@ -100,7 +119,7 @@ enum { TR_START = 0, TR_W_ISSUED, TR_PDL, TR_FIRST_FULL, TR_MMA_ISSUED, TR_DONE,
        TR_PREFETCHED, TR_ARRIVED, TR_ITER0, TR_EXIT, TR_PART, TR_ENTRY };
 
 struct GemmSmem {
-  int stages, stage_bytes, ring_bytes, part_off, recv_off, in_off, bar_off, total;
+  int stages, stage_bytes, ring_bytes, f8_off, part_off, recv_off, in_off, bar_off, total;
 };
 
 // Shared memory of one GEMM CTA: a ring of `stages` stages, each a 128x64
@@ -110,18 +129,21 @@ struct GemmSmem {
 // the receive buffer [cs * per][128] of the cluster reduction; the
 // epilogue's per-token inputs [per][128] (residual rows or RoPE cos/sin);
 // mbarriers.
-__host__ __device__ inline GemmSmem gemm_smem_layout(int stages, int n_mma, int cs, int T, bool with_in = true) {
+__host__ __device__ inline GemmSmem gemm_smem_layout(int stages, int n_mma, int cs, int T, bool with_in = true,
+                                                     bool f8 = false) {
   GemmSmem s;
   const int per = (T + cs - 1) / cs;
   s.stages = stages;
   s.stage_bytes = 16384 + n_mma * 128;
   s.ring_bytes = stages * s.stage_bytes;
+  s.f8_off = s.ring_bytes;   // FP8 weights: the E4M3 box of each stage, 8 KB, before widening
+  const int core = s.ring_bytes + (f8 ? stages * 8192 : 0);
   const int part_bytes = n_mma * 512;
   s.part_off = 0;   // the partial tile overlays the ring: every MMA has completed when it is written
-  s.recv_off = s.ring_bytes > part_bytes ? s.ring_bytes : part_bytes;
+  s.recv_off = core > part_bytes ? core : part_bytes;
   s.in_off = s.recv_off + cs * per * 512;   // [per][128] fp32 epilogue inputs of the owned tokens
   s.bar_off = s.in_off + (with_in ? per * 512 : 0);   // GU reads no per-token epilogue inputs
-  s.total = s.bar_off + (2 * stages + 2) * 8 + 16 + 1024;   // barriers, TMEM slot, alignment slack
+  s.total = s.bar_off + (3 * stages + 2) * 8 + 16 + 1024;   // barriers, TMEM slot, alignment slack
   return s;
 }
 
@@ -172,7 +194,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
   __shared__ float rs_s[kMaxOwn];
   const int n_mma = a.n_mma;
   const int cs = gridDim.x;
-  const GemmSmem L = gemm_smem_layout(a.stages, n_mma, cs, a.T, MODE != GM_GU);
+  const bool f8 = (MODE == GM_GU || MODE == GM_DOWN) && a.wt8 != nullptr;
+  const GemmSmem L = gemm_smem_layout(a.stages, n_mma, cs, a.T, MODE != GM_GU, f8);
   // every CTA of the grid sees the same values, so a refusal is uniform across each cluster
   if (dynamic_smem_size() < (uint32_t)L.total || a.kslice < 64 || (a.kslice & 63) || a.stages < 1 || n_mma > 256 ||
       (n_mma & 15) || a.T > n_mma || cs > 16 || (a.T + cs - 1) / cs > kMaxOwn) {
@@ -193,13 +216,17 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
   float* recv = (float*)(base + L.recv_off);           // [cs][per][128] partials of the tokens I own
   uint64_t* full = (uint64_t*)(base + L.bar_off);      // weight + activation boxes landed
   uint64_t* empty = full + NS;                         // the stage's MMAs completed
-  uint64_t* done = empty + NS;                         // all MMAs completed
+  uint64_t* conv = empty + NS;                         // FP8: the stage's weights widened to bf16
+  uint64_t* done = conv + NS;                          // all MMAs completed
   uint64_t* rbar = done + 1;                           // all partials of my tokens landed
   uint32_t* tmem_slot = (uint32_t*)(rbar + 1);
   const uint32_t ncols = (uint32_t)tmem_cols_for(n_mma);
   const uint32_t act_box_bytes = (uint32_t)n_mma * 128u;
   // this CTA's first weight box and first activation box
   const __nv_bfloat16* wsrc = a.wt + ((size_t)(a.w_tile0 + nt) * (a.K >> 6) + (k0 >> 6)) * 8192;
+  const uint8_t* wsrc8 = f8 ? a.wt8 + ((size_t)(a.w_tile0 + nt) * (a.K >> 6) + (k0 >> 6)) * 8192 : nullptr;
+  uint8_t* f8s = base + L.f8_off;                      // FP8 staging, 8 KB per stage
+  const uint32_t wbox_bytes = f8 ? 8192u : 16384u;
   const __nv_bfloat16* asrc = a.act + (size_t)(k0 >> 6) * n_mma * 64;
   unsigned long long* trace = a.trace ? a.trace + ((size_t)blockIdx.y * gridDim.x + blockIdx.x) * kTraceRow : nullptr;
   if (trace && threadIdx.x == 0) trace[TR_START] = ptx::globaltimer();
@@ -208,6 +235,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
     for (int i = 0; i < NS; ++i) {
       ptx::mbar_init(&full[i], 2);
       ptx::mbar_init(&empty[i], 1);
+      ptx::mbar_init(&conv[i], kEpiWarps);
     }
     ptx::mbar_init(done, 1);
     ptx::mbar_init(rbar, 1);
@@ -225,8 +253,9 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
     if (lane == 0) {
       pol = ptx::policy_evict_first();
       for (int b = 0; b < first; ++b) {
-        ptx::mbar_expect_tx(&full[b], 16384u);
-        ptx::bulk_load_hint(base + b * L.stage_bytes, wsrc + (size_t)b * 8192, 16384u, &full[b], pol);
+        ptx::mbar_expect_tx(&full[b], wbox_bytes);
+        if (f8) ptx::bulk_load_hint(f8s + b * 8192, wsrc8 + (size_t)b * 8192, 8192u, &full[b], pol);
+        else ptx::bulk_load_hint(base + b * L.stage_bytes, wsrc + (size_t)b * 8192, 16384u, &full[b], pol);
       }
       if (trace) trace[TR_W_ISSUED] = ptx::globaltimer();
     } else if (lane == 2 && a.pf) {
@@ -266,8 +295,9 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
           atomicOr(a.status, RTV_DEV_TIMEOUT);
           break;
         }
-        ptx::mbar_expect_tx(&full[s], 16384u);
-        ptx::bulk_load_hint(base + s * L.stage_bytes, wsrc + (size_t)b * 8192, 16384u, &full[s], pol);
+        ptx::mbar_expect_tx(&full[s], wbox_bytes);
+        if (f8) ptx::bulk_load_hint(f8s + s * 8192, wsrc8 + (size_t)b * 8192, 8192u, &full[s], pol);
+        else ptx::bulk_load_hint(base + s * L.stage_bytes, wsrc + (size_t)b * 8192, 16384u, &full[s], pol);
       }
     } else if (lane == 1) {
       ptx::pdl_wait();
@@ -286,9 +316,10 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
     // ---- MMA issue: one thread ----
     if (lane == 0) {
       const uint32_t idesc = ptx::idesc_bf16_f32(128, n_mma);
+      uint64_t* ready = f8 ? conv : full;   // FP8: the converters have seen the stage land and widened it
       for (int b = 0; b < nbox; ++b) {
         const int s = b % NS, u = b / NS;
-        if (!ptx::mbar_wait(&full[s], u & 1, a.timeout_ns)) {
+        if (!ptx::mbar_wait(&ready[s], u & 1, a.timeout_ns)) {
           atomicOr(a.status, RTV_DEV_TIMEOUT);
           break;
         }
@@ -349,6 +380,30 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
       for (int j2 = 0; j2 < n_wt; ++j2) sst += a.ssp[(size_t)(t_own0 + tid) * n_wt + j2];
       rs_s[tid] = rsqrtf(sst / (float)a.w + a.eps);
     }
+    // FP8 weights: per-row scales of this lane's features, and the widening
+    // of every stage's E4M3 box into the bf16 operand tile while the MMAs run
+    float2 ws1 = make_float2(1.f, 1.f), ws2 = make_float2(1.f, 1.f);
+    if (f8) {
+      ws1 = *reinterpret_cast<const float2*>(a.wscale + nt * 128 + f0);
+      ws2 = *reinterpret_cast<const float2*>(a.wscale + nt * 128 + 64 + f0);
+      for (int b = 0; b < nbox; ++b) {
+        const int s = b % NS, u = b / NS;
+        if (!ptx::mbar_wait(&full[s], u & 1, a.timeout_ns)) {
+          atomicOr(a.status, RTV_DEV_TIMEOUT);
+          break;
+        }
+        const uint8_t* src = f8s + s * 8192;          // [128 rows][64 codes]
+        uint8_t* dst = base + s * L.stage_bytes;       // [128 rows][64 bf16], 128-byte swizzle
+        for (int q = tid; q < 1024; q += kEpiThreads) {
+          const int r = q >> 3, c = q & 7;             // 8 codes -> one 16-byte chunk
+          const uint2 codes = *reinterpret_cast<const uint2*>(src + r * 64 + c * 8);
+          *reinterpret_cast<uint4*>(dst + r * 128 + ((c ^ (r & 7)) << 4)) = e4m3x8_to_bf16x8(codes);
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&conv[s]);
+      }
+    }
     if (!ptx::mbar_wait(done, 0, a.timeout_ns)) atomicOr(a.status, RTV_DEV_TIMEOUT);
     ptx::tc_fence_after();
     if (trace && tid == 0) trace[TR_DONE] = ptx::globaltimer();
@@ -408,6 +463,12 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
         x1.y += u1.y;
         x2.x += u2.x;
         x2.y += u2.y;
+      }
+      if (f8) {   // per-row scale of the FP8 weights (the split-K sum is linear in it)
+        x1.x *= ws1.x;
+        x1.y *= ws1.y;
+        x2.x *= ws2.x;
+        x2.y *= ws2.y;
       }
       if (MODE == GM_O || MODE == GM_DOWN) {
         // residual add, then the next norm's bf16 input and this tile's sum of squares
@@ -1257,6 +1318,26 @@ __global__ void pack_tiled_kernel(const __nv_bfloat16* __restrict__ src, __nv_bf
     *reinterpret_cast<uint4*>(d + ts_offset(r & 127, 8 * i, 128)) = s[i];
 }
 
+// FP8 weights: row r of the packed matrix is row idx[r] (or r) of a [rows][K]
+// E4M3 matrix, in 128-row tiles of [K/64] boxes [128][64] bytes (the
+// converters add the swizzle when they widen a box to bf16).
+__global__ void pack_tiled8_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst,
+                                   const int* __restrict__ idx, int rows, int K) {
+  const int r = blockIdx.x;
+  if (r >= rows) return;
+  const uint8_t* s = src + (size_t)(idx ? idx[r] : r) * K;
+  uint8_t* d = dst + (size_t)(r >> 7) * (K >> 6) * 8192 + (size_t)(r & 127) * 64;
+  for (int i = threadIdx.x; i < K / 16; i += blockDim.x) {
+    const int k = 16 * i;
+    *reinterpret_cast<uint4*>(d + (size_t)(k >> 6) * 8192 + (k & 63)) = *reinterpret_cast<const uint4*>(s + k);
+  }
+}
+
+__global__ void gather_f32_kernel(const float* __restrict__ src, float* __restrict__ dst, const int* __restrict__ idx,
+                                  int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) dst[i] = src[idx ? idx[i] : i];
+}
+
 // [rows][cols] -> [cols][rows]
 __global__ void transpose_bf16_kernel(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst,
                                       int rows, int cols) {
@@ -1277,6 +1358,9 @@ struct GemmPlan {
 struct FastPath {
   __nv_bfloat16 *w_qkv = nullptr, *w_o = nullptr, *w_gu = nullptr, *w_down = nullptr;
   __nv_bfloat16 *w_aiT = nullptr, *w_spT = nullptr;
+  bool mlp_f8 = false;                                      // gate/up/down in FP8 E4M3
+  uint8_t *w_gu8 = nullptr, *w_down8 = nullptr;             // their tiled codes, all layers
+  float *gu_s = nullptr, *down_s = nullptr;                 // per-row scales, packed row order, all layers
   __nv_bfloat16 *qb = nullptr, *ksb = nullptr, *vsb = nullptr, *ob = nullptr, *mb = nullptr, *hb = nullptr;
   float* ssp = nullptr;
   // attention partial rows [Gmax][Hq][16][64][D] (the tensor-core kernel
@@ -1320,7 +1404,7 @@ int round_up(int x, int m) { return (x + m - 1) / m * m; }
 // that does), otherwise one (the ring the deepest that fits the whole shared
 // memory); a cluster size is only usable as far as its clusters fit.  Ties
 // go to the smaller cluster (less reduction traffic).
-GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T, bool with_in) {
+GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T, bool with_in, bool f8 = false) {
   GemmPlan best;
   best.n_tiles = N / 128;
   double best_cost = 1e30;
@@ -1329,7 +1413,7 @@ GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T, bool with
     if (K % (cs * 64)) break;
     if ((T + cs - 1) / cs > 160) continue;   // tokens per rank (kMaxOwn in the kernel)
     const int nbox = K / cs / 64;
-    auto total = [&](int st) { return gemm_smem_layout(st, n_mma, cs, T, with_in).total; };
+    auto total = [&](int st) { return gemm_smem_layout(st, n_mma, cs, T, with_in, f8).total; };
     int stages = nbox;
     while (stages > 1 && total(stages) > fp->smem_cap) --stages;
     int per_sm = 2;
@@ -1670,11 +1754,18 @@ rtv_status fast_load(rtv_ctx* ctx, const rtv_tensor*, int) {
     fp->allocs.push_back(*p);
     return true;
   };
+  fp->mlp_f8 = k.mlp_dtype == RTV_FP8_E4M3;
   if (!(alloc((void**)&fp->w_qkv, Lh * nq * w * 2) && alloc((void**)&fp->w_o, (size_t)Lh * w * Q * 2) &&
-        alloc((void**)&fp->w_gu, Lh * ngu * w * 2) && alloc((void**)&fp->w_down, (size_t)Lh * w * F * 2) &&
         alloc((void**)&fp->w_aiT, (size_t)k.action_dim * w * 2) &&
         alloc((void**)&fp->w_spT, (size_t)k.state_dim * w * 2)))
     return RTV_ERR_OOM;
+  if (fp->mlp_f8) {
+    if (!(alloc((void**)&fp->w_gu8, Lh * ngu * w) && alloc((void**)&fp->w_down8, (size_t)Lh * w * F) &&
+          alloc((void**)&fp->gu_s, Lh * ngu * 4) && alloc((void**)&fp->down_s, (size_t)Lh * w * 4)))
+      return RTV_ERR_OOM;
+  } else if (!(alloc((void**)&fp->w_gu, Lh * ngu * w * 2) && alloc((void**)&fp->w_down, (size_t)Lh * w * F * 2))) {
+    return RTV_ERR_OOM;
+  }
   // row orders of the packed tiles: a QKV tile holds the RoPE pairs (d, d + D/2)
   // of one head; a gate/up tile holds 64 gate rows and the matching 64 up rows
   std::vector<int> iq(nq), igu(ngu);
@@ -1693,10 +1784,17 @@ rtv_status fast_load(rtv_ctx* ctx, const rtv_tensor*, int) {
     const LayerW& Lw = ctx->W.layers[l];
     pack_tiled_kernel<<<(int)nq, 128>>>((const __nv_bfloat16*)Lw.qkv, fp->w_qkv + (size_t)l * nq * w, d_iq,
                                         (int)nq, w);
-    pack_tiled_kernel<<<(int)ngu, 128>>>((const __nv_bfloat16*)Lw.gu, fp->w_gu + (size_t)l * ngu * w, d_igu,
-                                         (int)ngu, w);
     pack_tiled_kernel<<<w, 128>>>((const __nv_bfloat16*)Lw.o, fp->w_o + (size_t)l * w * Q, nullptr, w, Q);
-    pack_tiled_kernel<<<w, 128>>>((const __nv_bfloat16*)Lw.down, fp->w_down + (size_t)l * w * F, nullptr, w, F);
+    if (fp->mlp_f8) {
+      pack_tiled8_kernel<<<(int)ngu, 128>>>((const uint8_t*)Lw.gu, fp->w_gu8 + (size_t)l * ngu * w, d_igu, (int)ngu, w);
+      pack_tiled8_kernel<<<w, 128>>>((const uint8_t*)Lw.down, fp->w_down8 + (size_t)l * w * F, nullptr, w, F);
+      gather_f32_kernel<<<32, 256>>>(Lw.gu_s, fp->gu_s + (size_t)l * ngu, d_igu, (int)ngu);
+      gather_f32_kernel<<<4, 256>>>(Lw.down_s, fp->down_s + (size_t)l * w, nullptr, w);
+    } else {
+      pack_tiled_kernel<<<(int)ngu, 128>>>((const __nv_bfloat16*)Lw.gu, fp->w_gu + (size_t)l * ngu * w, d_igu,
+                                           (int)ngu, w);
+      pack_tiled_kernel<<<w, 128>>>((const __nv_bfloat16*)Lw.down, fp->w_down + (size_t)l * w * F, nullptr, w, F);
+    }
   }
   transpose_bf16_kernel<<<64, 256>>>((const __nv_bfloat16*)ctx->W.ai_w, fp->w_aiT, w, k.action_dim);
   transpose_bf16_kernel<<<64, 256>>>((const __nv_bfloat16*)ctx->W.sp_w, fp->w_spT, w, k.state_dim);
@@ -1756,8 +1854,8 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
   const int nq = Q + 2 * KV;
   const GemmPlan p_qkv = plan_gemm(fp, nq, w, n_mma, T, true);
   const GemmPlan p_o = plan_gemm(fp, w, Q, n_mma, T, true);
-  const GemmPlan p_gu = plan_gemm(fp, 2 * F, w, n_mma, T, false);
-  const GemmPlan p_dn = plan_gemm(fp, w, F, n_mma, T, true);
+  const GemmPlan p_gu = plan_gemm(fp, 2 * F, w, n_mma, T, false, fp->mlp_f8);
+  const GemmPlan p_dn = plan_gemm(fp, w, F, n_mma, T, true, fp->mlp_f8);
   const int nk = P + S;
   const int nchunk = attn_chunks(fp, nk, k.n_q_heads * G);
   if (!(p_qkv.valid && p_o.valid && p_gu.valid && p_dn.valid) ||
@@ -1896,24 +1994,28 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     a.act = fp->ob;
     a.K = Q;
     a.w_tile0 = l * w / 128;
-    a.pf = (const uint8_t*)(fp->w_gu + (size_t)l * 2 * F * w);
-    a.pf_bytes = (unsigned long long)2 * F * w * 2;
+    a.pf = fp->mlp_f8 ? fp->w_gu8 + (size_t)l * 2 * F * w : (const uint8_t*)(fp->w_gu + (size_t)l * 2 * F * w);
+    a.pf_bytes = (unsigned long long)2 * F * w * (fp->mlp_f8 ? 1 : 2);
     a.g_next = Lw.g_mlp;
     if (e == cudaSuccess) e = launch_gemm<GM_O>(a, p_o, st);
 
     a = base;
     a.trace = tr(l, 2);
     a.wt = fp->w_gu;
+    a.wt8 = fp->mlp_f8 ? fp->w_gu8 : nullptr;
+    a.wscale = fp->mlp_f8 ? fp->gu_s + (size_t)l * 2 * F : nullptr;
     a.act = fp->hb;
     a.K = w;
     a.w_tile0 = l * 2 * F / 128;
-    a.pf = (const uint8_t*)(fp->w_down + (size_t)l * w * F);
-    a.pf_bytes = (unsigned long long)w * F * 2;
+    a.pf = fp->mlp_f8 ? fp->w_down8 + (size_t)l * w * F : (const uint8_t*)(fp->w_down + (size_t)l * w * F);
+    a.pf_bytes = (unsigned long long)w * F * (fp->mlp_f8 ? 1 : 2);
     if (e == cudaSuccess) e = launch_gemm<GM_GU>(a, p_gu, st);
 
     a = base;
     a.trace = tr(l, 3);
     a.wt = fp->w_down;
+    a.wt8 = fp->mlp_f8 ? fp->w_down8 : nullptr;
+    a.wscale = fp->mlp_f8 ? fp->down_s + (size_t)l * w : nullptr;
     a.act = fp->mb;
     a.K = F;
     a.w_tile0 = l * w / 128;

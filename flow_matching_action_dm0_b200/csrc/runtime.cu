@@ -259,7 +259,8 @@ rtv_status rtv_create(const rtv_expert_config* cfg_in, int cuda_device, rtv_ctx*
     return RTV_ERR_ARG;
   if (k.dtype != RTV_F32 && k.dtype != RTV_BF16) return RTV_ERR_ARG;
   if (k.mlp_dtype == RTV_SAME) k.mlp_dtype = k.dtype;
-  if (k.mlp_dtype != k.dtype) return RTV_ERR_UNSUPPORTED;
+  // FP8 E4M3 MLP weights ride on bf16 activations (tensor-core path only)
+  if (k.mlp_dtype != k.dtype && !(k.mlp_dtype == RTV_FP8_E4M3 && k.dtype == RTV_BF16)) return RTV_ERR_UNSUPPORTED;
   if (k.suffix_mask != RTV_MASK_BIDIR && k.suffix_mask != RTV_MASK_PI0_BLOCK) return RTV_ERR_ARG;
   if (!(k.rms_eps >= 0.f) || !(k.rope_theta >= 0.f)) return RTV_ERR_ARG;
   if (k.barrier_timeout_ns <= 0) k.barrier_timeout_ns = 100000000LL;
@@ -320,6 +321,7 @@ rtv_status rtv_create(const rtv_expert_config* cfg_in, int cuda_device, rtv_ctx*
     const bool want_simt = env && strcmp(env, "simt") == 0;
     if (!want_simt) s = fast_create(ctx);
   }
+  if (s == RTV_OK && k.mlp_dtype == RTV_FP8_E4M3 && !ctx->use_fast) s = RTV_ERR_UNSUPPORTED;   // no SIMT FP8
   if (s != RTV_OK) {
     rtv_destroy(ctx);
     return s;
@@ -368,10 +370,17 @@ rtv_status rtv_load_expert(rtv_ctx* ctx, const rtv_tensor* params, int n_params)
     slots[p + "k_proj.w"] = Slot{{KV, w}, md, nullptr, (size_t)Q * w * e, &L.qkv, qkv_bytes};
     slots[p + "v_proj.w"] = Slot{{KV, w}, md, nullptr, (size_t)(Q + KV) * w * e, &L.qkv, qkv_bytes};
     mat(p + "o_proj.w", w, Q, &L.o);
-    const size_t gu_bytes = (size_t)2 * F * w * e;
-    slots[p + "gate_proj.w"] = Slot{{F, w}, md, nullptr, 0, &L.gu, gu_bytes};
-    slots[p + "up_proj.w"] = Slot{{F, w}, md, nullptr, (size_t)F * w * e, &L.gu, gu_bytes};
-    mat(p + "down_proj.w", w, F, &L.down);
+    const int mdt = k.mlp_dtype;
+    const size_t em = dtype_size(mdt);
+    const size_t gu_bytes = (size_t)2 * F * w * em;
+    slots[p + "gate_proj.w"] = Slot{{F, w}, mdt, nullptr, 0, &L.gu, gu_bytes};
+    slots[p + "up_proj.w"] = Slot{{F, w}, mdt, nullptr, (size_t)F * w * em, &L.gu, gu_bytes};
+    slots[p + "down_proj.w"] = Slot{{w, F}, mdt, &L.down, 0, nullptr, 0};
+    if (mdt == RTV_FP8_E4M3) {
+      slots[p + "gate_proj.s"] = Slot{{F}, RTV_F32, nullptr, 0, (void**)&L.gu_s, (size_t)2 * F * 4};
+      slots[p + "up_proj.s"] = Slot{{F}, RTV_F32, nullptr, (size_t)F * 4, (void**)&L.gu_s, (size_t)2 * F * 4};
+      vec(p + "down_proj.s", w, &L.down_s);
+    }
   }
 
   // validate every entry first: nothing is allocated on a bad table

@@ -16,8 +16,10 @@ namespace rtv {
 struct LayerW {
   void* qkv = nullptr;    // [Q+2KV][w]   q rows, then k rows, then v rows (simt layout)
   void* o = nullptr;      // [w][Q]
-  void* gu = nullptr;     // [2F][w]      gate rows, then up rows (simt layout)
+  void* gu = nullptr;     // [2F][w]      gate rows, then up rows (simt layout; E4M3 codes with an FP8 MLP)
   void* down = nullptr;   // [w][F]
+  float* gu_s = nullptr;  // [2F] per-row scales of gate then up (FP8 MLP only)
+  float* down_s = nullptr;   // [w] per-row scales of down (FP8 MLP only)
   float* g_attn = nullptr;
   float* g_mlp = nullptr;
 };

@@ -84,7 +84,10 @@ typedef enum {
  * dtype (RTV_F32 or RTV_BF16) is the storage and tensor-core input type of
  * the weight matrices and of the prefix KV; biases and norm gains are fp32.
  * mlp_dtype: RTV_SAME, or RTV_FP8_E4M3 for gate/up/down weights stored in
- * E4M3 with one fp32 scale per output row ([DM0.5] 6.3).
+ * E4M3 with one fp32 scale per output row ([DM0.5] 6.3), with dtype
+ * RTV_BF16 only (bf16 activations, fp32 accumulation; the E4M3 values are
+ * widened to bf16 exactly).  A shape the tensor-core path does not take
+ * returns RTV_ERR_UNSUPPORTED from rtv_create for an FP8 MLP.
  * rope_theta 0 disables rotary embedding.  barrier_timeout_ns bounds every
  * device-side wait (0 = library default, 100 ms).
  */
