@@ -46,7 +46,8 @@ Where the pages are silent the plainest reading is taken:
   R6 GELU tanh approximation in the gated MLP.
   R7 biases only on state_proj, action_in/out_proj and the time MLP.
   R8 only the H action rows produce velocity; the state row is discarded.
-  R10 FP8 MLP (BASELINE's FP8 configuration): gate/up/down given as E4M3
+  R10 FP8 MLP (the pi0-fp8mlp workload; [DM0.5] 6.3 names FP8 E4M3 for the
+     gate/up/down GEMMs): gate/up/down given as E4M3
      codes with one fp32 scale per output row; W = decode(code) * scale,
      everything else unchanged (bf16 activations, fp32 accumulation on the
      device; fp64 here).
@@ -90,7 +91,7 @@ def e4m3_decode(codes: np.ndarray) -> np.ndarray:
 def to_f64(weights: Dict[str, np.ndarray]) -> Dict[str, np.ndarray]:
     """fp64 values of the given parameters.  A matrix given as FP8 E4M3 codes
     (uint8) is decoded and multiplied row by row by its fp32 scale (the
-    tensor of the same name ending in ".s"): BASELINE's FP8 MLP storage,
+    tensor of the same name ending in ".s"): the FP8 MLP storage,
     one scale per output channel."""
     out: Dict[str, np.ndarray] = {}
     for k, v in weights.items():

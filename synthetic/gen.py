@@ -17,7 +17,7 @@ bf16 inputs are produced by round-to-nearest-even of the float32 draw; both
 the oracle and the CUDA path receive the same rounded values.
 
 In an FP8-MLP workload the gate/up/down matrices are *given* in FP8 E4M3
-storage with one fp32 scale per output row (BASELINE's FP8 configuration):
+storage with one fp32 scale per output row (the pi0-fp8mlp workload):
 the float32 draw of a row is divided by scale = max|row| / 448 and rounded to
 the nearest E4M3 value (ties to even).  The codes and scales are the inputs;
 what an E4M3 code means is decoded by each side on its own.
