@@ -53,7 +53,7 @@ typedef enum {
   RTV_ERR_OOM = 5,         /* device allocation failed                        */
   RTV_ERR_TIMEOUT = 6,     /* a device-side bounded wait gave up              */
   RTV_ERR_NUMERIC = 7,     /* non-finite value detected on the device        */
-  RTV_ERR_UNSUPPORTED = 8  /* valid request this build does not implement     */
+  RTV_ERR_UNSUPPORTED = 8  /* valid request the library does not implement   */
 } rtv_status;
 
 typedef enum { RTV_F32 = 0, RTV_BF16 = 1, RTV_FP8_E4M3 = 2, RTV_SAME = 3 } rtv_dtype;
