@@ -109,6 +109,7 @@ struct GemmArgs {
   unsigned long long* trace;  // optional phase stamps [cta][16] (globaltimer ns), or nullptr
   long long timeout_ns;
   int T, n_mma, kslice, stages, w, S, Hq, Hkv, D, F, K, w_tile0;
+  int tt;                     // token rows per CTA (a multiple of 16, <= 256); blockIdx.z picks the tile
   float eps;
 };
 
@@ -192,13 +193,19 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
   extern __shared__ uint8_t smem_raw[];
   constexpr int kMaxOwn = 160;   // tokens one rank reduces and finishes
   __shared__ float rs_s[kMaxOwn];
-  const int n_mma = a.n_mma;
+  // Token tiling: blockIdx.z takes token rows [t0, t0 + n_mma) of the tiled
+  // activation layout, which has n_rows rows per 64-column block; T of them are
+  // real tokens.
+  const int n_rows = a.n_mma;
+  const int t0 = (int)blockIdx.z * a.tt;
+  const int n_mma = min(a.tt, n_rows - t0);
+  const int T = min(a.T - t0, n_mma);
   const int cs = gridDim.x;
   const bool f8 = (MODE == GM_GU || MODE == GM_DOWN) && a.wt8 != nullptr;
-  const GemmSmem L = gemm_smem_layout(a.stages, n_mma, cs, a.T, MODE != GM_GU, f8);
-  // every CTA of the grid sees the same values, so a refusal is uniform across each cluster
+  const GemmSmem L = gemm_smem_layout(a.stages, n_mma, cs, T, MODE != GM_GU, f8);
+  // every CTA of a cluster sees the same values, so a refusal is uniform across it
   if (dynamic_smem_size() < (uint32_t)L.total || a.kslice < 64 || (a.kslice & 63) || a.stages < 1 || n_mma > 256 ||
-      (n_mma & 15) || a.T > n_mma || cs > 16 || (a.T + cs - 1) / cs > kMaxOwn) {
+      n_mma < 16 || (n_mma & 15) || (n_rows & 15) || T < 1 || T > n_mma || cs > 16 || (T + cs - 1) / cs > kMaxOwn) {
     if (threadIdx.x == 0) atomicOr(a.status, RTV_DEV_BOUNDS);
     return;
   }
@@ -209,9 +216,9 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
   const int nbox = a.kslice >> 6;
   const int NS = L.stages;
   const int k0 = (int)rank * a.kslice;
-  const int per = (a.T + cs - 1) / cs;                 // tokens owned by each rank in the reduction
-  const int t_own0 = (int)rank * per;
-  const int n_own = max(0, min(a.T, t_own0 + per) - t_own0);
+  const int per = (T + cs - 1) / cs;                   // tokens owned by each rank in the reduction
+  const int t_own0 = (int)rank * per;                  // (tile-local)
+  const int n_own = max(0, min(T, t_own0 + per) - t_own0);
   float* part = (float*)(base + L.part_off);           // [n_mma][128] this CTA's partial sums
   float* recv = (float*)(base + L.recv_off);           // [cs][per][128] partials of the tokens I own
   uint64_t* full = (uint64_t*)(base + L.bar_off);      // weight + activation boxes landed
@@ -227,8 +234,9 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
   const uint8_t* wsrc8 = f8 ? a.wt8 + ((size_t)(a.w_tile0 + nt) * (a.K >> 6) + (k0 >> 6)) * 8192 : nullptr;
   uint8_t* f8s = base + L.f8_off;                      // FP8 staging, 8 KB per stage
   const uint32_t wbox_bytes = f8 ? 8192u : 16384u;
-  const __nv_bfloat16* asrc = a.act + (size_t)(k0 >> 6) * n_mma * 64;
-  unsigned long long* trace = a.trace ? a.trace + ((size_t)blockIdx.y * gridDim.x + blockIdx.x) * kTraceRow : nullptr;
+  const __nv_bfloat16* asrc = a.act + ((size_t)(k0 >> 6) * n_rows + t0) * 64;
+  const size_t trace_row = ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+  unsigned long long* trace = (a.trace && trace_row < 512) ? a.trace + trace_row * kTraceRow : nullptr;
   if (trace && threadIdx.x == 0) trace[TR_START] = ptx::globaltimer();
 
   if (threadIdx.x == 0) {
@@ -309,7 +317,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
           break;
         }
         ptx::mbar_expect_tx(&full[s], act_box_bytes);
-        ptx::bulk_load(base + s * L.stage_bytes + 16384, asrc + (size_t)b * n_mma * 64, act_box_bytes, &full[s]);
+        ptx::bulk_load(base + s * L.stage_bytes + 16384, asrc + (size_t)b * n_rows * 64, act_box_bytes, &full[s]);
       }
     }
   } else if (warp == 1) {
@@ -357,12 +365,12 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
     if (MODE == GM_O || MODE == GM_DOWN) {
       for (int c = tid; c < n_own * 32; c += kEpiThreads) {
         const int tl = c >> 5, ch = c & 31;
-        ptx::cp_async_16(in_a + (uint32_t)(c * 16), a.h + (size_t)(t_own0 + tl) * a.w + nt * 128 + ch * 4);
+        ptx::cp_async_16(in_a + (uint32_t)(c * 16), a.h + (size_t)(t0 + t_own0 + tl) * a.w + nt * 128 + ch * 4);
       }
     } else if (rope) {
       for (int c = tid; c < n_own * 32; c += kEpiThreads) {
         const int tl = c >> 5, ch = c & 31;   // chunks 0-15: cos, 16-31: sin (64 floats each)
-        const int s = (t_own0 + tl) % a.S;
+        const int s = (t0 + t_own0 + tl) % a.S;
         const float* src = (ch < 16 ? a.rope_cs : a.rope_sn) + (size_t)s * hd + dq0 + (ch & 15) * 4;
         ptx::cp_async_16(in_a + (uint32_t)(c * 16), src);
       }
@@ -377,7 +385,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
     }
     if ((MODE == GM_QKV || MODE == GM_GU) && tid < n_own) {
       float sst = 0.f;
-      for (int j2 = 0; j2 < n_wt; ++j2) sst += a.ssp[(size_t)(t_own0 + tid) * n_wt + j2];
+      for (int j2 = 0; j2 < n_wt; ++j2) sst += a.ssp[(size_t)(t0 + t_own0 + tid) * n_wt + j2];
       rs_s[tid] = rsqrtf(sst / (float)a.w + a.eps);
     }
     // FP8 weights: per-row scales of this lane's features, and the widening
@@ -432,7 +440,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
     if (tid < cs) {   // one lane per destination rank
       const int r = tid;
       const uint32_t part_a = ptx::smem_u32(part), recv_a = ptx::smem_u32(recv), rbar_a = ptx::smem_u32(rbar);
-      const int o0 = r * per, no = max(0, min(a.T, o0 + per) - o0);
+      const int o0 = r * per, no = max(0, min(T, o0 + per) - o0);
       if (no > 0)
         bulk_copy_to_rank(ptx::mapa(recv_a + (uint32_t)(rank * per * 512), (uint32_t)r),
                           part_a + (uint32_t)(o0 * 512), (uint32_t)(no * 512), ptx::mapa(rbar_a, (uint32_t)r));
@@ -453,7 +461,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
     const int ew = warp - 2;
 #pragma unroll 1
     for (int tl = ew; tl < n_own; tl += kEpiWarps) {
-      const int t = t_own0 + tl;
+      const int t = t0 + t_own0 + tl;   // global token row
       float2 x1 = make_float2(0.f, 0.f), x2 = make_float2(0.f, 0.f);
       for (int qr = 0; qr < cs; ++qr) {
         const float* rr = recv + (qr * per + tl) * 128;
@@ -484,9 +492,9 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
           sq = fmaf(h2.x, h2.x, sq);
           sq = fmaf(h2.y, h2.y, sq);
           sq = warp_sum(sq);
-          *reinterpret_cast<uint32_t*>(a.hb + ts_offset(t, n1, n_mma)) =
+          *reinterpret_cast<uint32_t*>(a.hb + ts_offset(t, n1, n_rows)) =
               ptx::pack_bf16x2(h1.x * (1.f + gn1.x), h1.y * (1.f + gn1.y));
-          *reinterpret_cast<uint32_t*>(a.hb + ts_offset(t, n2, n_mma)) =
+          *reinterpret_cast<uint32_t*>(a.hb + ts_offset(t, n2, n_rows)) =
               ptx::pack_bf16x2(h2.x * (1.f + gn2.x), h2.y * (1.f + gn2.y));
           if (lane == 0) a.ssp[(size_t)t * n_wt + nt] = sq;
         }
@@ -497,7 +505,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
         x2.x *= rs;
         x2.y *= rs;
         if (MODE == GM_GU) {
-          *reinterpret_cast<uint32_t*>(a.m + ts_offset(t, nt * 64 + f0, n_mma)) =
+          *reinterpret_cast<uint32_t*>(a.m + ts_offset(t, nt * 64 + f0, n_rows)) =
               ptx::pack_bf16x2(gelu_tanh(x1.x) * x2.x, gelu_tanh(x1.y) * x2.y);
         } else {
           const int g = t / a.S, s = t - g * a.S;
@@ -615,8 +623,9 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
   const __nv_bfloat16* svh = a.sv + ((size_t)g * a.Hkv + kvh) * a.S * D;
 
   unsigned long long* trace =
-      a.trace ? a.trace + (((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * kTraceRow
-              : nullptr;
+      (a.trace && ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x < 512)
+          ? a.trace + (((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * kTraceRow
+          : nullptr;
   if (trace && tid == 0) trace[0] = ptx::globaltimer();
   ptx::pdl_launch_dependents();
 
@@ -905,8 +914,9 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const AttnTcArgs a) {
   const int kvh = (2 * hp * a.Hkv) / a.Hq;
   const bool suffix_tile = rank == ntp;
   unsigned long long* trace =
-      a.trace ? a.trace + (((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * kTraceRow
-              : nullptr;
+      (a.trace && ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x < 512)
+          ? a.trace + (((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * kTraceRow
+          : nullptr;
   if (trace && tid == 0) trace[0] = ptx::globaltimer();
   if (tid == 0) {
     for (int i = 0; i < 4; ++i) ptx::mbar_init(&bars[i], 1);
@@ -1352,6 +1362,7 @@ __global__ void transpose_bf16_kernel(const __nv_bfloat16* __restrict__ src, __n
 // ===========================================================================
 struct GemmPlan {
   int n_tiles = 0, cs = 1, kslice = 0, stages = 1, smem = 0;
+  int n_tt = 1;   // token tiles (grid z)
   bool valid = false;
 };
 
@@ -1404,9 +1415,11 @@ int round_up(int x, int m) { return (x + m - 1) / m * m; }
 // that does), otherwise one (the ring the deepest that fits the whole shared
 // memory); a cluster size is only usable as far as its clusters fit.  Ties
 // go to the smaller cluster (less reduction traffic).
-GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T, bool with_in, bool f8 = false) {
+GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T, bool with_in, bool f8 = false,
+                   int n_tt = 1) {
   GemmPlan best;
   best.n_tiles = N / 128;
+  best.n_tt = n_tt;
   double best_cost = 1e30;
   constexpr double kFixedBoxes = 8.0;   // a wave's fixed latency, in MMA boxes (~3 us)
   for (int cs = 1; cs <= fp->max_cluster; cs <<= 1) {
@@ -1423,10 +1436,10 @@ GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T, bool with
       while (stages > 1 && total(stages) > kDynSmemMax) --stages;
       if (total(stages) > kDynSmemMax) continue;
     }
-    const int ctas = best.n_tiles * cs;
+    const int ctas = best.n_tiles * cs * n_tt;
     const int fit = per_sm * std::max(1, fp->gemm_fit_large[cs]);   // clusters resident at once
     const int waves = std::max((ctas + per_sm * fp->num_sms - 1) / (per_sm * fp->num_sms),
-                               (best.n_tiles + fit - 1) / fit);
+                               (best.n_tiles * n_tt + fit - 1) / fit);
     const double cost = waves * (kFixedBoxes + nbox);
     if (cost < best_cost) {
       best_cost = cost;
@@ -1444,7 +1457,7 @@ template <int MODE>
 cudaError_t launch_gemm(const GemmArgs& a, const GemmPlan& pl, cudaStream_t st) {
   auto kern = gemm_tc_kernel<MODE>;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(pl.cs, pl.n_tiles, 1);
+  cfg.gridDim = dim3(pl.cs, pl.n_tiles, pl.n_tt);
   cfg.blockDim = dim3(kGemmThreads, 1, 1);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = st;
@@ -1592,7 +1605,7 @@ rtv_status fast_create(rtv_ctx* ctx) {
   const int n_mma_max = round_up(ctx->Gmax * S, 16);
   const bool shape_ok = k.dtype == RTV_BF16 && (k.head_dim == 128 || k.head_dim == 256) && k.width % 128 == 0 &&
                         k.width <= 1024 && k.mlp_dim % 128 == 0 && (ctx->Q % 128) == 0 && S <= 64 &&
-                        k.action_dim <= 64 && k.state_dim <= 64 && n_mma_max <= 256;
+                        k.action_dim <= 64 && k.state_dim <= 64 && n_mma_max > 0;
   if (!shape_ok) return RTV_OK;
   int dev = ctx->device;
   if (configure_gemm<GM_QKV>() != cudaSuccess || configure_gemm<GM_O>() != cudaSuccess ||
@@ -1850,12 +1863,18 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
   FastPath* fp = ctx->fast;
   const rtv_expert_config& k = ctx->cfg;
   const int S = ctx->S, T = G * S, w = k.width, F = k.mlp_dim, D = k.head_dim, Q = ctx->Q, KV = ctx->KV;
-  const int n_mma = round_up(T, 16);
+  const int n_mma = round_up(T, 16);   // rows of the tiled activation layout
+  // Token tiles, one per grid z.  Up to 208 rows stay one tile; beyond, tiles
+  // of about 128 rows keep a CTA's fp32 partial tile and reduction buffers
+  // (512 bytes per token row each) within shared memory.
+  const int n_tt = n_mma <= 208 ? 1 : (n_mma + 127) / 128;
+  const int tt = round_up((n_mma + n_tt - 1) / n_tt, 16);
+  const int T_tile = std::min(T, tt);
   const int nq = Q + 2 * KV;
-  const GemmPlan p_qkv = plan_gemm(fp, nq, w, n_mma, T, true);
-  const GemmPlan p_o = plan_gemm(fp, w, Q, n_mma, T, true);
-  const GemmPlan p_gu = plan_gemm(fp, 2 * F, w, n_mma, T, false, fp->mlp_f8);
-  const GemmPlan p_dn = plan_gemm(fp, w, F, n_mma, T, true, fp->mlp_f8);
+  const GemmPlan p_qkv = plan_gemm(fp, nq, w, tt, T_tile, true, false, n_tt);
+  const GemmPlan p_o = plan_gemm(fp, w, Q, tt, T_tile, true, false, n_tt);
+  const GemmPlan p_gu = plan_gemm(fp, 2 * F, w, tt, T_tile, false, fp->mlp_f8, n_tt);
+  const GemmPlan p_dn = plan_gemm(fp, w, F, tt, T_tile, true, fp->mlp_f8, n_tt);
   const int nk = P + S;
   const int nchunk = attn_chunks(fp, nk, k.n_q_heads * G);
   if (!(p_qkv.valid && p_o.valid && p_gu.valid && p_dn.valid) ||
@@ -1891,6 +1910,7 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
   base.timeout_ns = k.barrier_timeout_ns;
   base.T = T;
   base.n_mma = n_mma;
+  base.tt = tt;
   base.w = w;
   base.S = S;
   base.Hq = k.n_q_heads;
@@ -1953,11 +1973,11 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
   const bool tracing = fp->trace_armed && fp->trace != nullptr;
   fp->trace_armed = false;
   if (tracing) {
-    fp->trace_ctas[0] = p_qkv.n_tiles * p_qkv.cs;
-    fp->trace_ctas[1] = p_o.n_tiles * p_o.cs;
-    fp->trace_ctas[2] = p_gu.n_tiles * p_gu.cs;
-    fp->trace_ctas[3] = p_dn.n_tiles * p_dn.cs;
-    fp->trace_ctas[4] = tc_att ? (ntp + 1) * (k.n_q_heads / 2) * G : nchunk * k.n_q_heads * G;
+    fp->trace_ctas[0] = std::min(512, p_qkv.n_tiles * p_qkv.cs * n_tt);
+    fp->trace_ctas[1] = std::min(512, p_o.n_tiles * p_o.cs * n_tt);
+    fp->trace_ctas[2] = std::min(512, p_gu.n_tiles * p_gu.cs * n_tt);
+    fp->trace_ctas[3] = std::min(512, p_dn.n_tiles * p_dn.cs * n_tt);
+    fp->trace_ctas[4] = std::min(512, tc_att ? (ntp + 1) * (k.n_q_heads / 2) * G : nchunk * k.n_q_heads * G);
   }
   auto tr = [&](int l, int i) -> unsigned long long* {
     return (tracing && l == 0) ? fp->trace + (size_t)i * 512 * kTraceRow : nullptr;

@@ -114,6 +114,15 @@ def test_pi0_bf16_batch_two_matches_oracle(cuda_ok):
     assert bf16_tolerance_ok(got, ref)
 
 
+def test_pi0_bf16_batch_sixteen_token_tiles(cuda_ok):
+    """16 chunks = 816 token rows: four token tiles of the projections (the
+    MMA N is at most 256), sixteen suffix groups in the attention."""
+    cfg = get_config("pi0-bf16", n_layers=2, prefix_len=200)
+    got, ref, path = run_denoise(cfg, batch=16, n_steps=2)
+    assert path == "tcgen05"
+    assert bf16_tolerance_ok(got, ref), (rel_l2(got, ref), np.max(np.abs(got - ref)))
+
+
 def test_repeat_calls_are_bitwise_identical(cuda_ok):
     cfg = get_config("pi0-bf16", n_layers=2)
     ex, _, _ = build_expert(cfg)

@@ -50,6 +50,12 @@ def test_fp8_mlp_batch_four_matches_oracle(cuda_ok):
     assert bf16_tolerance_ok(got, ref), (rel_l2(got, ref), np.max(np.abs(got - ref)))
 
 
+def test_fp8_mlp_batch_sixteen_matches_oracle(cuda_ok):
+    cfg = get_config("pi0-fp8mlp", n_layers=2, batch=16)
+    got, ref = _denoise(cfg, 2, batch=16)
+    assert bf16_tolerance_ok(got, ref), (rel_l2(got, ref), np.max(np.abs(got - ref)))
+
+
 def test_fp8_mlp_verify_distances_match_oracle(cuda_ok):
     cfg = get_config("pi0-fp8mlp", n_layers=2)
     ex, weights, kv = build_expert(cfg)
