@@ -1,7 +1,9 @@
 """Oracle package (TEST INFRASTRUCTURE): plain fp64 CPU statement of the method.
 
 Only tests/, __graft_entry__.smoke() and bench.py's CPU-baseline and
-reference legs may import it.  See ``oracle.expert`` for the cited passages.
+reference legs may import it.  See ``oracle.expert`` (the action expert and
+FLASH verification) and ``oracle.draft`` (the FLASH draft model and round)
+for the cited passages.
 """
 
-from . import expert  # noqa: F401
+from . import draft, expert  # noqa: F401

@@ -7,15 +7,18 @@ attention, no time embedding, no Euler step), so the oracle and the CUDA
 path can both use it without sharing any computation.
 """
 
-from .configs import CONFIGS, ExpertShape, get_config  # noqa: F401
+from .configs import CONFIGS, DRAFTS, DraftShape, ExpertShape, get_config, get_draft_config  # noqa: F401
 from .gen import (  # noqa: F401
     bf16_bits_to_f32,
     e4m3_encode,
     f32_to_bf16_bits,
+    draft_weight_names,
     make_draft,
+    make_draft_weights,
     make_noise,
     make_prefix_kv,
     make_state,
+    make_visual_tokens,
     make_weights,
     round_to_bf16,
     weight_names,

@@ -15,6 +15,16 @@ Names:
                  + 48 text), 1 state token + 50 action tokens of dim 32.
   pi0-verify     FLASH verification on the pi0-bf16 expert, taus 0.2/0.5/0.8.
   pi0-fp8mlp     pi0-bf16 with FP8 E4M3 MLP weights and a 560-token prefix.
+
+Draft models ("Realtime-VLA FLASH" sec. 03.1: one Gemma block and a linear
+action head, about 110M parameters, learnable action queries reading the
+current image features in one forward pass):
+  draft-tiny     width-256 block in fp32, 8 queries, 7-dim actions, 64
+                 visual tokens.
+  flash-draft    Gemma-2B-width block (width 2048, 8 q / 1 kv heads,
+                 head_dim 256, GeGLU 16384: 110.1M block parameters), 50
+                 queries of 32-dim actions over the 768 image tokens (3 views
+                 x 256) of the pi0-bf16 observation, bf16.
 """
 
 from __future__ import annotations
@@ -94,6 +104,63 @@ PI0_VERIFY = PI0_BF16.with_(name="pi0-verify")
 PI0_FP8MLP = PI0_BF16.with_(name="pi0-fp8mlp", mlp_dtype="fp8_e4m3", prefix_len=560)
 
 CONFIGS = {c.name: c for c in (TINY_FP32, PI0_BF16, PI0_VERIFY, PI0_FP8MLP)}
+
+
+@dataclass(frozen=True)
+class DraftShape:
+    """A FLASH draft model: one Gemma block over [visual tokens ; action
+    queries] and a linear action head on the query rows."""
+    name: str
+    width: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    mlp_dim: int
+    n_queries: int          # H, rows of the candidate chunk
+    action_dim: int         # A
+    n_vis: int              # V, visual tokens of one observation
+    batch: int = 1
+    dtype: str = "f32"      # storage/MMA type of matrices and visual tokens
+    rms_eps: float = 1e-6
+    rope_theta: float = 10000.0
+    weight_std: float = 0.02
+    seed: int = 0
+
+    @property
+    def q_dim(self) -> int:
+        return self.n_q_heads * self.head_dim
+
+    @property
+    def kv_dim(self) -> int:
+        return self.n_kv_heads * self.head_dim
+
+    def with_(self, **kw) -> "DraftShape":
+        return replace(self, **kw)
+
+    def block_params(self) -> int:
+        w, f = self.width, self.mlp_dim
+        return w * (self.q_dim + 2 * self.kv_dim) + self.q_dim * w + 3 * w * f + 2 * w
+
+    def params(self) -> int:
+        return self.block_params() + self.n_queries * self.width + self.action_dim * (self.width + 1)
+
+
+TINY_DRAFT = DraftShape(
+    name="draft-tiny", width=256, n_q_heads=4, n_kv_heads=1, head_dim=64, mlp_dim=1024, n_queries=8,
+    action_dim=7, n_vis=64, dtype="f32",
+)
+
+FLASH_DRAFT = DraftShape(
+    name="flash-draft", width=2048, n_q_heads=8, n_kv_heads=1, head_dim=256, mlp_dim=16384, n_queries=50,
+    action_dim=32, n_vis=768, dtype="bf16",
+)
+
+DRAFTS = {c.name: c for c in (TINY_DRAFT, FLASH_DRAFT)}
+
+
+def get_draft_config(name: str, **overrides) -> DraftShape:
+    cfg = DRAFTS[name]
+    return cfg.with_(**overrides) if overrides else cfg
 
 
 def get_config(name: str, **overrides) -> ExpertShape:

@@ -30,7 +30,7 @@ from typing import Dict, List, Tuple
 
 import numpy as np
 
-from .configs import ExpertShape
+from .configs import DraftShape, ExpertShape
 
 
 def _rng(seed: int, name: str) -> np.random.Generator:
@@ -189,3 +189,57 @@ def make_draft(cfg: ExpertShape, n_switch: int = 0, seed: int | None = None) -> 
         g[r:] = -sign0
     d[:, cfg.gripper] = g
     return d
+
+
+# ---------------------------------------------------------------------------
+# FLASH draft model (one Gemma block + linear action head over learnable
+# action queries and the image features)
+# ---------------------------------------------------------------------------
+
+def draft_weight_names(dcfg: DraftShape) -> List[Tuple[str, Tuple[int, ...]]]:
+    """(name, shape) of every draft-model parameter, matrices as [out][in]."""
+    w, f = dcfg.width, dcfg.mlp_dim
+    return [
+        ("action_queries", (dcfg.n_queries, w)),
+        ("attn_norm.g", (w,)),
+        ("q_proj.w", (dcfg.q_dim, w)),
+        ("k_proj.w", (dcfg.kv_dim, w)),
+        ("v_proj.w", (dcfg.kv_dim, w)),
+        ("o_proj.w", (w, dcfg.q_dim)),
+        ("mlp_norm.g", (w,)),
+        ("gate_proj.w", (f, w)),
+        ("up_proj.w", (f, w)),
+        ("down_proj.w", (w, f)),
+        ("action_head.w", (dcfg.action_dim, w)),
+        ("action_head.b", (dcfg.action_dim,)),
+    ]
+
+
+def make_draft_weights(dcfg: DraftShape, seed: int | None = None) -> Dict[str, np.ndarray]:
+    """Draft-model parameters as float32 arrays: matrices, gains and the head
+    bias ~ N(0, 0.02); the action queries ~ N(0, 1) (the scale of the visual
+    tokens they are read beside).  In a "bf16" draft every weight matrix holds
+    bf16-representable values; the queries stay float32 (they seed the fp32
+    residual stream)."""
+    seed = dcfg.seed if seed is None else seed
+    ws: Dict[str, np.ndarray] = {}
+    for name, shape in draft_weight_names(dcfg):
+        std = 1.0 if name == "action_queries" else dcfg.weight_std
+        a = _normal(seed, "draft." + name, shape, std)
+        if dcfg.dtype == "bf16" and len(shape) == 2 and name != "action_queries":
+            a = round_to_bf16(a)
+        ws[name] = a
+    return ws
+
+
+def make_visual_tokens(dcfg: DraftShape, batch: int | None = None, n_vis: int | None = None,
+                       seed: int | None = None) -> np.ndarray:
+    """Image features [B][V][w] ~ N(0,1) (bf16 values in a bf16 draft): the
+    stand-in for the vision encoder's projected tokens of one observation."""
+    seed = dcfg.seed if seed is None else seed
+    b = dcfg.batch if batch is None else batch
+    v = dcfg.n_vis if n_vis is None else n_vis
+    x = _normal(seed, "visual_tokens", (b, v, dcfg.width), 1.0)
+    if dcfg.dtype == "bf16":
+        x = round_to_bf16(x)
+    return x

@@ -91,3 +91,29 @@ def velocity(W, cfg, x_t, state, t, prefix_k, prefix_v):
 
     hf = F.rms_norm(h[:, 1:], (w,), weight=1.0 + _t(W["final_norm.g"]), eps=eps)
     return F.linear(hf, _t(W["action_out_proj.w"]), _t(W["action_out_proj.b"])).numpy()
+
+
+def draft(W, dcfg, vis):
+    """Candidate chunks [B][H][A] of the FLASH draft model for vis [B][V][w]:
+    the queries are concatenated after the visual tokens of every batch
+    element and one block runs over the batched sequences."""
+    vis = _t(vis)
+    b, v_len, w = vis.shape
+    h_len = dcfg.n_queries
+    n = v_len + h_len
+    hq, hkv, d = dcfg.n_q_heads, dcfg.n_kv_heads, dcfg.head_dim
+    eps = dcfg.rms_eps
+    x = torch.cat([vis, _t(W["action_queries"]).expand(b, h_len, w)], dim=1)     # [B, n, w]
+    pos = torch.arange(n)
+    u = F.rms_norm(x, (w,), weight=1.0 + _t(W["attn_norm.g"]), eps=eps)
+    q = rope_complex(F.linear(u, _t(W["q_proj.w"])).view(b, n, hq, d), pos, dcfg.rope_theta)
+    k = rope_complex(F.linear(u, _t(W["k_proj.w"])).view(b, n, hkv, d), pos, dcfg.rope_theta)
+    v = F.linear(u, _t(W["v_proj.w"])).view(b, n, hkv, d)
+    rep = hq // hkv
+    o = F.scaled_dot_product_attention(q.transpose(1, 2), k.transpose(1, 2).repeat_interleave(rep, dim=1),
+                                       v.transpose(1, 2).repeat_interleave(rep, dim=1))
+    h = x + F.linear(o.transpose(1, 2).reshape(b, n, hq * d), _t(W["o_proj.w"]))
+    u = F.rms_norm(h, (w,), weight=1.0 + _t(W["mlp_norm.g"]), eps=eps)
+    gate = F.gelu(F.linear(u, _t(W["gate_proj.w"])), approximate="tanh")
+    h = h + F.linear(gate * F.linear(u, _t(W["up_proj.w"])), _t(W["down_proj.w"]))
+    return F.linear(h[:, v_len:], _t(W["action_head.w"]), _t(W["action_head.b"])).numpy()
