@@ -54,6 +54,8 @@ def parse_args(argv=None):
                     help="override the workload's layer count (profiling runs on smaller captures only; "
                          "the JSON line then names the reduced depth)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-round", action="store_true",
+                    help="skip the FLASH draft model / dual-path round measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds of the oracle sample")
     ap.add_argument("--trace", action="store_true",
                     help="print the library's phase stamps of layer 0 of the first Euler step (no timing)")
@@ -320,6 +322,11 @@ def run_ours(args, info):
         v_ms.append(v0.elapsed_time(v1))
     verify_us = float(np.median(v_ms)) * 1000.0
 
+    round_info = None
+    if info.world == 1 and not args.no_round and cfg.batch == 1 and args.layers <= 0 and \
+            (cfg.chunk_len, cfg.action_dim) == (50, 32):
+        round_info = measure_round(ex, cfg, noise_d, state_d, stream, dev, K)
+
     launches_per_call = ex.kernels_per_call(n)
     path = ex.path
     ex.close()
@@ -368,6 +375,8 @@ def run_ours(args, info):
                    "note": "one FLASH verification (len(taus) suffixes in one expert evaluation + decision), "
                            "host buffers, device time per call (median)"},
     }
+    if round_info is not None:
+        line["flash_round"] = round_info
     if info.world == 1 and not args.no_cpu_baseline:
         per_step_s, k = oracle_step_seconds(cfg, args.cpu_seconds)
         line["cpu_baseline"] = {
@@ -375,6 +384,90 @@ def run_ours(args, info):
             "sample": f"{k} single Euler steps of the {args.workload} chunk (fp64 numpy oracle, median), "
                       f"scaled x{n} to one chunk"}
     print(json.dumps(line), flush=True)
+
+
+def draft_bytes(dcfg) -> int:
+    """Algorithmic bytes of one draft forward: the block's and head's weights,
+    the queries, the image features read, and their keys/values written and
+    read back once."""
+    e = 2 if dcfg.dtype == "bf16" else 4
+    w = dcfg.width
+    kv = dcfg.n_vis * 2 * dcfg.kv_dim * e
+    return (dcfg.block_params() - 2 * w) * e + 2 * w * 4 + dcfg.action_dim * (w * e + 4) + \
+        dcfg.n_queries * w * 4 + dcfg.n_vis * w * e + 2 * kv
+
+
+def measure_round(ex, cfg, noise, state, stream, dev, K):
+    """FLASH draft model (the flash-draft workload: one Gemma-2B-width block,
+    110M parameters, 768 image tokens) and one dual-path round on the
+    expert: device time of the draft forward, and of a whole round in each
+    branch (CUDA events around the call; the host reads the verdict in
+    between, so the span includes that gap)."""
+    import torch
+
+    from flow_matching_action_dm0_b200 import DraftModel, flash_round
+    from synthetic import f32_to_bf16_bits, get_draft_config, make_draft_weights, make_visual_tokens
+
+    dcfg = get_draft_config("flash-draft")
+    dw = make_draft_weights(dcfg)
+    # accept branch: the head's gripper row is zeroed and its bias made
+    # positive, so the random draft holds the gripper still (no switch)
+    dw_acc = dict(dw)
+    dw_acc["action_head.w"] = dw["action_head.w"].copy()
+    dw_acc["action_head.w"][cfg.gripper] = 0.0
+    dw_acc["action_head.b"] = dw["action_head.b"].copy()
+    dw_acc["action_head.b"][cfg.gripper] = 0.5
+    vis = make_visual_tokens(dcfg)
+    vis_d = torch.from_numpy(f32_to_bf16_bits(vis).view(np.int16)).view(torch.bfloat16).cuda(dev)
+    out_d = torch.empty((1, dcfg.n_queries, dcfg.action_dim), dtype=torch.float32, device=dev)
+    taus = tuple(cfg.taus)
+    res = {"draft_workload": "flash-draft", "draft_params": dcfg.params(), "n_vis": dcfg.n_vis, "taus": list(taus),
+           "n_steps": cfg.n_steps}
+    for branch, weights, delta in (("accept", dw_acc, 1e6), ("fallback", dw, 0.05)):
+        dm = DraftModel(dcfg, device=dev, max_batch=1)
+        dm.load(weights)
+        for _ in range(3):
+            dm.forward(vis_d, out_d, stream=stream)
+        torch.cuda.synchronize(dev)
+        if branch == "accept":
+            d_ms = []
+            for _ in range(max(10, min(K, 50))):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                dm.forward(vis_d, out_d, stream=stream)
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                d_ms.append(e0.elapsed_time(e1))
+            draft_us = float(np.median(d_ms)) * 1000.0
+            nbytes = draft_bytes(dcfg)
+            res["draft_us"] = draft_us
+            res["draft_kernels"] = dm.kernels_per_call(dcfg.n_vis, 1)
+            res["draft_roofline"] = {"bound": "hbm", "algorithmic_bytes": nbytes,
+                                     "achieved": nbytes / (draft_us * 1e-6) / 1e9, "unit": "GB/s"}
+        r = None
+        for _ in range(2):
+            r = flash_round(ex, dm, vis_d[0], noise[0], state[0], taus, delta, cfg.gripper, cfg.n_steps,
+                            stream=stream)
+        r_ms = []
+        for _ in range(max(5, min(K, 20))):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            r = flash_round(ex, dm, vis_d[0], noise[0], state[0], taus, delta, cfg.gripper, cfg.n_steps,
+                            stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            r_ms.append(e0.elapsed_time(e1))
+        res[f"round_{branch}_us"] = float(np.median(r_ms)) * 1000.0
+        res[f"round_{branch}_verdict"] = {"accepted_len": r.accepted_len, "flags": r.flags,
+                                          "used_full": r.used_full, "delta": delta}
+        s, bits = dm.status()
+        if s != 0:
+            raise RuntimeError(f"draft device status {bits:#x}")
+        dm.close()
+    res["note"] = ("accept branch = draft + verify + verdict read + draft copied out (gripper row of the random "
+                   "head zeroed, bias 0.5, delta 1e6); fallback branch = the same + 10-step denoise (random head, "
+                   "gripper switches); device time per round, median, CUDA events around the synchronous call")
+    return res
 
 
 def run_trace(args):

@@ -2,10 +2,12 @@
 
 The computation lives in ``librtv.so`` (CUDA, sm_100a; C ABI in
 ``include/rtv.h``).  This package holds the ctypes binding (``_lib``), a
-small handle class (``expert.ActionExpert``), the build script (``build``)
-and the replica plumbing for several GPUs (``replicas``).
+small handle class (``expert.ActionExpert``), the FLASH draft model and
+round (``draft.DraftModel``, ``draft.flash_round``), the build script
+(``build``) and the replica plumbing for several GPUs (``replicas``).
 """
 
 from . import _lib  # noqa: F401
 from ._lib import RtvError, load_library  # noqa: F401
+from .draft import DraftModel, flash_round, make_draft_config  # noqa: F401
 from .expert import ActionExpert, make_config  # noqa: F401

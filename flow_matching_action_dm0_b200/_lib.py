@@ -26,7 +26,9 @@ RTV_FLAG_ZERO_ACCEPT, RTV_FLAG_SWITCH, RTV_FLAG_SWITCH_IN_PREFIX = 1, 2, 4
 # Every symbol include/rtv.h declares (checked by the CPU test suite).
 EXPORTS = ("rtv_create", "rtv_load_expert", "rtv_set_prefix_kv", "rtv_denoise", "rtv_verify",
            "rtv_device_status", "rtv_last_error", "rtv_path_name", "rtv_graph_kernel_count", "rtv_destroy",
-           "rtv_set_prefix_kv_static")
+           "rtv_set_prefix_kv_static", "rtv_draft_create", "rtv_draft_load", "rtv_draft_forward", "rtv_flash_round",
+           "rtv_draft_device_status", "rtv_draft_last_error", "rtv_draft_path_name", "rtv_draft_kernel_count",
+           "rtv_draft_destroy")
 
 
 class rtv_expert_config(C.Structure):
@@ -36,6 +38,15 @@ class rtv_expert_config(C.Structure):
         ("chunk_len", C.c_int), ("max_prefix_len", C.c_int), ("max_batch", C.c_int), ("max_taus", C.c_int),
         ("dtype", C.c_int), ("mlp_dtype", C.c_int), ("suffix_mask", C.c_int),
         ("rms_eps", C.c_float), ("rope_theta", C.c_float), ("barrier_timeout_ns", C.c_longlong),
+    ]
+
+
+class rtv_draft_config(C.Structure):
+    _fields_ = [
+        ("width", C.c_int), ("n_q_heads", C.c_int), ("n_kv_heads", C.c_int), ("head_dim", C.c_int),
+        ("mlp_dim", C.c_int), ("n_queries", C.c_int), ("action_dim", C.c_int), ("max_vis", C.c_int),
+        ("max_batch", C.c_int), ("dtype", C.c_int), ("rms_eps", C.c_float), ("rope_theta", C.c_float),
+        ("barrier_timeout_ns", C.c_longlong),
     ]
 
 
@@ -79,8 +90,22 @@ def load_library(path: str = LIB_PATH):
     lib.rtv_graph_kernel_count.restype = I
     lib.rtv_destroy.argtypes = [P]
     lib.rtv_destroy.restype = None
+    lib.rtv_draft_create.argtypes = [C.POINTER(rtv_draft_config), I, C.POINTER(P)]
+    lib.rtv_draft_load.argtypes = [P, C.POINTER(rtv_tensor), I]
+    lib.rtv_draft_forward.argtypes = [P, P, I, I, P, P]
+    lib.rtv_flash_round.argtypes = [P, P, P, I, P, P, P, I, F, I, I, P, P, P, P, P]
+    lib.rtv_draft_device_status.argtypes = [P, U]
+    lib.rtv_draft_last_error.argtypes = [P]
+    lib.rtv_draft_last_error.restype = C.c_char_p
+    lib.rtv_draft_path_name.argtypes = [P]
+    lib.rtv_draft_path_name.restype = C.c_char_p
+    lib.rtv_draft_kernel_count.argtypes = [P, I, I]
+    lib.rtv_draft_kernel_count.restype = I
+    lib.rtv_draft_destroy.argtypes = [P]
+    lib.rtv_draft_destroy.restype = None
     for n in ("rtv_create", "rtv_load_expert", "rtv_set_prefix_kv", "rtv_set_prefix_kv_static", "rtv_denoise",
-              "rtv_verify", "rtv_device_status"):
+              "rtv_verify", "rtv_device_status", "rtv_draft_create", "rtv_draft_load", "rtv_draft_forward",
+              "rtv_flash_round", "rtv_draft_device_status"):
         getattr(lib, n).restype = I
     _lib = lib
     return lib
@@ -152,3 +177,61 @@ def rtv_graph_kernel_count(h, n: int, is_verify: bool = False) -> int:
 def rtv_destroy(h):
     if h:
         load_library().rtv_destroy(h)
+
+
+# draft model and FLASH round ------------------------------------------------
+
+def rtv_draft_create(cfg: rtv_draft_config, device: int = 0):
+    lib = load_library()
+    h = C.c_void_p()
+    s = lib.rtv_draft_create(C.byref(cfg), int(device), C.byref(h))
+    if s != RTV_OK:
+        raise RtvError(s, "rtv_draft_create failed")
+    return h
+
+
+def _dcheck(d, s):
+    if s != RTV_OK:
+        raise RtvError(s, load_library().rtv_draft_last_error(d).decode())
+    return s
+
+
+def rtv_draft_load(d, tensors):
+    arr = (rtv_tensor * len(tensors))(*tensors)
+    return _dcheck(d, load_library().rtv_draft_load(d, arr, len(tensors)))
+
+
+def rtv_draft_forward(d, vis_ptr: int, n_vis: int, batch: int, out_ptr: int, stream: int = 0):
+    return _dcheck(d, load_library().rtv_draft_forward(d, C.c_void_p(vis_ptr), int(n_vis), int(batch),
+                                                       C.c_void_p(out_ptr), C.c_void_p(stream)))
+
+
+def rtv_flash_round(h, d, vis_ptr, n_vis, noise_ptr, state_ptr, taus_ptr, n_taus, delta, gripper_dim, n_steps,
+                    out_ptr, acc_ptr, flags_ptr, used_full_ptr, stream: int = 0):
+    return _dcheck(d, load_library().rtv_flash_round(
+        h, d, C.c_void_p(vis_ptr), int(n_vis), C.c_void_p(noise_ptr), C.c_void_p(state_ptr), C.c_void_p(taus_ptr),
+        int(n_taus), C.c_float(delta), int(gripper_dim), int(n_steps), C.c_void_p(out_ptr), C.c_void_p(acc_ptr),
+        C.c_void_p(flags_ptr), C.c_void_p(used_full_ptr), C.c_void_p(stream)))
+
+
+def rtv_draft_device_status(d):
+    bits = C.c_uint(0)
+    s = load_library().rtv_draft_device_status(d, C.byref(bits))
+    return s, bits.value
+
+
+def rtv_draft_last_error(d) -> str:
+    return load_library().rtv_draft_last_error(d).decode()
+
+
+def rtv_draft_path_name(d) -> str:
+    return load_library().rtv_draft_path_name(d).decode()
+
+
+def rtv_draft_kernel_count(d, n_vis: int, batch: int) -> int:
+    return int(load_library().rtv_draft_kernel_count(d, int(n_vis), int(batch)))
+
+
+def rtv_draft_destroy(d):
+    if d:
+        load_library().rtv_draft_destroy(d)

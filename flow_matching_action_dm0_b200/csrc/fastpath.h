@@ -1,6 +1,7 @@
 // Tensor-core (tcgen05) path of the bf16 expert: interface used by the runtime.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "../../include/rtv.h"
@@ -25,6 +26,17 @@ rtv_status fast_step(rtv_ctx* ctx, int G, bool do_head, bool do_embed, float dt,
 // The expert's layers over G suffixes (residual stream ctx->h).
 rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, const float* rope_cs,
                        const float* rope_sn, cudaStream_t st);
+// Bare block (ctx->block_only), layer 0: keys and values of n_vis tokens per
+// batch element given as bf16 rows vis [batch][n_vis][width] (RMSNorm, K/V
+// projection, RoPE at positions 0..n_vis-1), written into the cached prefix,
+// whose tensor-core tiles are refreshed.  hb_vis (bf16, tiled over
+// round_up(batch*n_vis, 16) rows) and ssp_vis ([batch*n_vis][width/128]) are
+// scratch of the caller.
+rtv_status fast_block_prefix(rtv_ctx* ctx, const __nv_bfloat16* vis, int n_vis, int batch, __nv_bfloat16* hb_vis,
+                             float* ssp_vis, const float* rope_cs, const float* rope_sn, cudaStream_t st);
+// Bare block: residual stream of G suffixes set to rows[t % n_src_rows]
+// (fp32, [n_src_rows][width]) with the first norm's inputs.
+rtv_status fast_block_embed(rtv_ctx* ctx, const float* rows, int n_src_rows, int G, cudaStream_t st);
 void fast_destroy(rtv_ctx* ctx);
 // Diagnostic phase trace (only when the RTV_TRACE environment variable is set).
 void fast_arm_trace(rtv_ctx* ctx);

@@ -110,6 +110,8 @@ struct GemmArgs {
   long long timeout_ns;
   int T, n_mma, kslice, stages, w, S, Hq, Hkv, D, F, K, w_tile0;
   int tt;                     // token rows per CTA (a multiple of 16, <= 256); blockIdx.z picks the tile
+  int nt_base;                // first 128-row weight tile of the grid within the layer (QKV: K/V tiles only)
+  int kv_rows;                // row stride of ks / vs per (suffix, kv head) when qt is not set
   float eps;
 };
 
@@ -212,7 +214,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = ptx::cluster_ctarank();
-  const int nt = blockIdx.y;
+  const int nt = (int)blockIdx.y + a.nt_base;
   const int nbox = a.kslice >> 6;
   const int NS = L.stages;
   const int k0 = (int)rank * a.kslice;
@@ -537,8 +539,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
           } else {
             __nv_bfloat16* dst;
             if (hh < a.Hq) dst = a.q + ((size_t)t * a.Hq + hh) * a.D;
-            else if (hh < a.Hq + a.Hkv) dst = a.ks + (((size_t)g * a.Hkv + (hh - a.Hq)) * a.S + s) * a.D;
-            else dst = a.vs + (((size_t)g * a.Hkv + (hh - a.Hq - a.Hkv)) * a.S + s) * a.D;
+            else if (hh < a.Hq + a.Hkv) dst = a.ks + (((size_t)g * a.Hkv + (hh - a.Hq)) * a.kv_rows + s) * a.D;
+            else dst = a.vs + (((size_t)g * a.Hkv + (hh - a.Hq - a.Hkv)) * a.kv_rows + s) * a.D;
             *reinterpret_cast<uint32_t*>(dst + d1) = ptx::pack_bf16x2(y1.x, y1.y);
             *reinterpret_cast<uint32_t*>(dst + d2) = ptx::pack_bf16x2(y2.x, y2.y);
           }
@@ -1357,6 +1359,58 @@ __global__ void transpose_bf16_kernel(const __nv_bfloat16* __restrict__ src, __n
   }
 }
 
+// ---------------------------------------------------------------------------
+// Rows that enter a block from outside its residual stream (the draft
+// model's image features and action queries): the first norm's input
+// bf16(x * (1 + g)), tiled over n_rows token rows, and the sums of squares
+// of x per 128-feature tile; with h set, also x as the fp32 residual row.
+// Row t reads x row t % x_rows.  One CTA of 4 warps per row; warp j takes
+// the tiles j, j + 4, ...
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void load4_f32(const float* p, float v[4]) {
+  const float4 q = *reinterpret_cast<const float4*>(p);
+  v[0] = q.x;
+  v[1] = q.y;
+  v[2] = q.z;
+  v[3] = q.w;
+}
+__device__ __forceinline__ void load4_f32(const __nv_bfloat16* p, float v[4]) {
+  const uint2 q = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
+  v[0] = a.x;
+  v[1] = a.y;
+  v[2] = b.x;
+  v[3] = b.y;
+}
+
+template <typename XT>
+__global__ void __launch_bounds__(128) norm_input_kernel(const XT* __restrict__ x, int x_rows, float* __restrict__ h,
+                                                         const float* __restrict__ g, __nv_bfloat16* __restrict__ hb,
+                                                         float* __restrict__ ssp, int n_rows, int w) {
+  const int t = blockIdx.x;
+  const XT* xr = x + (size_t)(t % x_rows) * w;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_wt = w >> 7;
+  for (int j = warp; j < n_wt; j += 4) {
+    const int k = j * 128 + lane * 4;
+    float v[4];
+    load4_f32(xr + k, v);
+    float sq = v[0] * v[0];
+    sq = fmaf(v[1], v[1], sq);
+    sq = fmaf(v[2], v[2], sq);
+    sq = fmaf(v[3], v[3], sq);
+    sq = warp_sum(sq);
+    if (lane == 0) ssp[(size_t)t * n_wt + j] = sq;
+    if (h) *reinterpret_cast<float4*>(h + (size_t)t * w + k) = make_float4(v[0], v[1], v[2], v[3]);
+    const float4 gg = *reinterpret_cast<const float4*>(g + k);
+    uint2 packed;
+    packed.x = ptx::pack_bf16x2(v[0] * (1.f + gg.x), v[1] * (1.f + gg.y));
+    packed.y = ptx::pack_bf16x2(v[2] * (1.f + gg.z), v[3] * (1.f + gg.w));
+    *reinterpret_cast<uint2*>(hb + ts_offset(t, k, n_rows)) = packed;
+  }
+}
+
 // ===========================================================================
 // host side
 // ===========================================================================
@@ -1603,9 +1657,11 @@ rtv_status fast_create(rtv_ctx* ctx) {
   ctx->use_fast = false;
   const int S = ctx->S;
   const int n_mma_max = round_up(ctx->Gmax * S, 16);
+  // (the step kernel, which a bare block does not use, limits the width and
+  // the action and state sizes)
+  const bool step_ok = ctx->block_only || (k.width <= 1024 && k.action_dim <= 64 && k.state_dim <= 64);
   const bool shape_ok = k.dtype == RTV_BF16 && (k.head_dim == 128 || k.head_dim == 256) && k.width % 128 == 0 &&
-                        k.width <= 1024 && k.mlp_dim % 128 == 0 && (ctx->Q % 128) == 0 && S <= 64 &&
-                        k.action_dim <= 64 && k.state_dim <= 64 && n_mma_max > 0;
+                        k.mlp_dim % 128 == 0 && (ctx->Q % 128) == 0 && S <= 64 && step_ok && n_mma_max > 0;
   if (!shape_ok) return RTV_OK;
   int dev = ctx->device;
   if (configure_gemm<GM_QKV>() != cudaSuccess || configure_gemm<GM_O>() != cudaSuccess ||
@@ -1768,9 +1824,10 @@ rtv_status fast_load(rtv_ctx* ctx, const rtv_tensor*, int) {
     return true;
   };
   fp->mlp_f8 = k.mlp_dtype == RTV_FP8_E4M3;
-  if (!(alloc((void**)&fp->w_qkv, Lh * nq * w * 2) && alloc((void**)&fp->w_o, (size_t)Lh * w * Q * 2) &&
-        alloc((void**)&fp->w_aiT, (size_t)k.action_dim * w * 2) &&
-        alloc((void**)&fp->w_spT, (size_t)k.state_dim * w * 2)))
+  if (!(alloc((void**)&fp->w_qkv, Lh * nq * w * 2) && alloc((void**)&fp->w_o, (size_t)Lh * w * Q * 2)))
+    return RTV_ERR_OOM;
+  if (!ctx->block_only && !(alloc((void**)&fp->w_aiT, (size_t)k.action_dim * w * 2) &&
+                            alloc((void**)&fp->w_spT, (size_t)k.state_dim * w * 2)))
     return RTV_ERR_OOM;
   if (fp->mlp_f8) {
     if (!(alloc((void**)&fp->w_gu8, Lh * ngu * w) && alloc((void**)&fp->w_down8, (size_t)Lh * w * F) &&
@@ -1809,8 +1866,10 @@ rtv_status fast_load(rtv_ctx* ctx, const rtv_tensor*, int) {
       pack_tiled_kernel<<<w, 128>>>((const __nv_bfloat16*)Lw.down, fp->w_down + (size_t)l * w * F, nullptr, w, F);
     }
   }
-  transpose_bf16_kernel<<<64, 256>>>((const __nv_bfloat16*)ctx->W.ai_w, fp->w_aiT, w, k.action_dim);
-  transpose_bf16_kernel<<<64, 256>>>((const __nv_bfloat16*)ctx->W.sp_w, fp->w_spT, w, k.state_dim);
+  if (!ctx->block_only) {
+    transpose_bf16_kernel<<<64, 256>>>((const __nv_bfloat16*)ctx->W.ai_w, fp->w_aiT, w, k.action_dim);
+    transpose_bf16_kernel<<<64, 256>>>((const __nv_bfloat16*)ctx->W.sp_w, fp->w_spT, w, k.state_dim);
+  }
   cudaError_t e = cudaDeviceSynchronize();
   cudaFree(d_iq);
   cudaFree(d_igu);
@@ -1858,17 +1917,87 @@ rtv_status fast_step(rtv_ctx* ctx, int G, bool do_head, bool do_embed, float dt,
   return RTV_OK;
 }
 
+// Token tiles of a projection over n_mma tiled rows: up to 208 rows stay one
+// tile; beyond, tiles of about 128 rows keep a CTA's fp32 partial tile and
+// reduction buffers (512 bytes per token row each) within shared memory.
+void token_tiles(int n_mma, int* n_tt, int* tt) {
+  *n_tt = n_mma <= 208 ? 1 : (n_mma + 127) / 128;
+  *tt = round_up((n_mma + *n_tt - 1) / *n_tt, 16);
+}
+
+rtv_status fast_block_prefix(rtv_ctx* ctx, const __nv_bfloat16* vis, int n_vis, int batch, __nv_bfloat16* hb_vis,
+                             float* ssp_vis, const float* rope_cs, const float* rope_sn, cudaStream_t st) {
+  FastPath* fp = ctx->fast;
+  const rtv_expert_config& k = ctx->cfg;
+  const int w = k.width, D = k.head_dim, KV = ctx->KV;
+  const int T = batch * n_vis, n_mma = round_up(T, 16);
+  int n_tt = 1, tt = 16;
+  token_tiles(n_mma, &n_tt, &tt);
+  const LayerW& Lw = ctx->W.layers[0];
+  norm_input_kernel<__nv_bfloat16><<<T, 128, 0, st>>>(vis, T, nullptr, Lw.g_attn, hb_vis, ssp_vis, n_mma, w);
+  cudaError_t e = cudaGetLastError();
+  const GemmPlan p = plan_gemm(fp, 2 * KV, w, tt, std::min(T, tt), true, false, n_tt);
+  if (!p.valid) {
+    ctx->last_error = "no tensor-core split fits the visual-token projection";
+    return RTV_ERR_UNSUPPORTED;
+  }
+  // keys and values of the visual tokens: the K and V weight tiles of the
+  // layer (the q tiles are skipped), RoPE at positions 0..n_vis-1, written
+  // into the cached prefix [2][Bmax][Hkv][Pmax][D] of layer 0
+  const size_t kv_layer = (size_t)k.max_batch * k.n_kv_heads * k.max_prefix_len * D;
+  GemmArgs a{};
+  a.wt = fp->w_qkv;
+  a.act = hb_vis;
+  a.ssp = ssp_vis;
+  a.ks = (__nv_bfloat16*)ctx->prefix_kv;
+  a.vs = a.ks + kv_layer;
+  a.kv_rows = k.max_prefix_len;
+  a.rope_cs = rope_cs;
+  a.rope_sn = rope_sn;
+  a.status = ctx->status;
+  a.timeout_ns = k.barrier_timeout_ns;
+  a.T = T;
+  a.n_mma = n_mma;
+  a.tt = tt;
+  a.w = w;
+  a.S = n_vis;
+  a.Hq = k.n_q_heads;
+  a.Hkv = k.n_kv_heads;
+  a.D = D;
+  a.F = k.mlp_dim;
+  a.K = w;
+  a.w_tile0 = 0;
+  a.nt_base = ctx->Q / 128;
+  a.eps = k.rms_eps;
+  if (e == cudaSuccess) e = launch_gemm<GM_QKV>(a, p, st);
+  if (e != cudaSuccess) {
+    ctx->last_error = std::string("visual-token projection launch: ") + cudaGetErrorString(e);
+    return RTV_ERR_CUDA;
+  }
+  return fast_prefix_update(ctx, batch, n_vis, st);
+}
+
+rtv_status fast_block_embed(rtv_ctx* ctx, const float* rows, int n_src_rows, int G, cudaStream_t st) {
+  FastPath* fp = ctx->fast;
+  const int T = G * ctx->S;
+  norm_input_kernel<float><<<T, 128, 0, st>>>(rows, n_src_rows, ctx->h, ctx->W.layers[0].g_attn, fp->hb, fp->ssp,
+                                              round_up(T, 16), ctx->cfg.width);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    ctx->last_error = std::string("block input launch: ") + cudaGetErrorString(e);
+    return RTV_ERR_CUDA;
+  }
+  return RTV_OK;
+}
+
 rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, const float* rope_cs,
                        const float* rope_sn, cudaStream_t st) {
   FastPath* fp = ctx->fast;
   const rtv_expert_config& k = ctx->cfg;
   const int S = ctx->S, T = G * S, w = k.width, F = k.mlp_dim, D = k.head_dim, Q = ctx->Q, KV = ctx->KV;
   const int n_mma = round_up(T, 16);   // rows of the tiled activation layout
-  // Token tiles, one per grid z.  Up to 208 rows stay one tile; beyond, tiles
-  // of about 128 rows keep a CTA's fp32 partial tile and reduction buffers
-  // (512 bytes per token row each) within shared memory.
-  const int n_tt = n_mma <= 208 ? 1 : (n_mma + 127) / 128;
-  const int tt = round_up((n_mma + n_tt - 1) / n_tt, 16);
+  int n_tt = 1, tt = 16;               // token tiles, one per grid z
+  token_tiles(n_mma, &n_tt, &tt);
   const int T_tile = std::min(T, tt);
   const int nq = Q + 2 * KV;
   const GemmPlan p_qkv = plan_gemm(fp, nq, w, tt, T_tile, true, false, n_tt);
@@ -1911,6 +2040,7 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
   base.T = T;
   base.n_mma = n_mma;
   base.tt = tt;
+  base.kv_rows = S;
   base.w = w;
   base.S = S;
   base.Hq = k.n_q_heads;

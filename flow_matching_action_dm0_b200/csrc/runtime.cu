@@ -18,6 +18,40 @@
 
 using namespace rtv;
 
+namespace rtv {
+
+// The layers of a context over G suffixes (residual stream ctx->h, T = G*S
+// rows), SIMT kernels.  [DM0.5] 5.2: RMSNorm -> q/k/v -> RoPE -> attention
+// over [prefix ; own suffix] -> o_proj + residual -> RMSNorm -> GeGLU MLP +
+// residual.
+template <typename WT>
+void simt_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, const float* rope_cs, const float* rope_sn,
+                 cudaStream_t st) {
+  const rtv_expert_config& k = ctx->cfg;
+  const int S = ctx->S, T = G * S, w = k.width, F = k.mlp_dim;
+  const int Q = ctx->Q, KV = ctx->KV, D = k.head_dim;
+  const size_t kv_layer = (size_t)k.max_batch * k.n_kv_heads * k.max_prefix_len * D;
+  for (int l = 0; l < k.n_layers; ++l) {
+    const LayerW& L = ctx->W.layers[l];
+    const WT* pk = (const WT*)ctx->prefix_kv + (size_t)(2 * l) * kv_layer;
+    const WT* pv = (const WT*)ctx->prefix_kv + (size_t)(2 * l + 1) * kv_layer;
+    launch_rmsnorm(ctx->h, L.g_attn, ctx->u, T, w, k.rms_eps, st);
+    launch_linear<WT>(ctx->u, w, (const WT*)L.qkv, nullptr, ctx->qkv, Q + 2 * KV, T, Q + 2 * KV, w, EPI_STORE, st);
+    launch_rope_split(ctx->qkv, rope_cs, rope_sn, ctx->q, ctx->ks, ctx->vs, T, S, k.n_q_heads, k.n_kv_heads, D, st);
+    launch_attention_simt<WT>(ctx->q, pk, pv, ctx->ks, ctx->vs, ctx->o, T, S, P, k.max_prefix_len, k.n_q_heads,
+                              k.n_kv_heads, D, prefix_batch_stride, k.suffix_mask, st);
+    launch_linear<WT>(ctx->o, Q, (const WT*)L.o, nullptr, ctx->h, w, T, w, Q, EPI_ADD, st);
+    launch_rmsnorm(ctx->h, L.g_mlp, ctx->u, T, w, k.rms_eps, st);
+    launch_linear<WT>(ctx->u, w, (const WT*)L.gu, nullptr, ctx->gu, 2 * F, T, 2 * F, w, EPI_STORE, st);
+    launch_geglu(ctx->gu, ctx->m, T, F, st);
+    launch_linear<WT>(ctx->m, F, (const WT*)L.down, nullptr, ctx->h, w, T, w, F, EPI_ADD, st);
+  }
+}
+template void simt_layers<float>(rtv_ctx*, int, int, int, const float*, const float*, cudaStream_t);
+template void simt_layers<__nv_bfloat16>(rtv_ctx*, int, int, int, const float*, const float*, cudaStream_t);
+
+}  // namespace rtv
+
 namespace {
 
 rtv_status fail(rtv_ctx* c, rtv_status s, const std::string& msg) {
@@ -70,34 +104,15 @@ struct DeviceGuard {
   }
 };
 
-// ---------------------------------------------------------------------------
 // SIMT forward of the expert over G suffixes (token rows T = G*S) and the
 // output head.  Used for the fp32 expert and, on request, the bf16 expert.
-// ---------------------------------------------------------------------------
 template <typename WT>
 void simt_expert(rtv_ctx* ctx, int G, int P, const float* c, int c_stride, int state_stride, int prefix_batch_stride,
                  const float* rope_cs, const float* rope_sn, cudaStream_t st) {
   const rtv_expert_config& k = ctx->cfg;
-  const int S = ctx->S, T = G * S, w = k.width, F = k.mlp_dim;
-  const int Q = ctx->Q, KV = ctx->KV, D = k.head_dim;
   launch_embed<WT>(ctx->x, ctx->state, state_stride, (const WT*)ctx->W.sp_w, ctx->W.sp_b, (const WT*)ctx->W.ai_w,
-                   ctx->W.ai_b, c, c_stride, ctx->h, G, w, S, k.action_dim, k.state_dim, st);
-  const size_t kv_layer = (size_t)k.max_batch * k.n_kv_heads * k.max_prefix_len * D;
-  for (int l = 0; l < k.n_layers; ++l) {
-    const LayerW& L = ctx->W.layers[l];
-    const WT* pk = (const WT*)ctx->prefix_kv + (size_t)(2 * l) * kv_layer;
-    const WT* pv = (const WT*)ctx->prefix_kv + (size_t)(2 * l + 1) * kv_layer;
-    launch_rmsnorm(ctx->h, L.g_attn, ctx->u, T, w, k.rms_eps, st);
-    launch_linear<WT>(ctx->u, w, (const WT*)L.qkv, nullptr, ctx->qkv, Q + 2 * KV, T, Q + 2 * KV, w, EPI_STORE, st);
-    launch_rope_split(ctx->qkv, rope_cs, rope_sn, ctx->q, ctx->ks, ctx->vs, T, S, k.n_q_heads, k.n_kv_heads, D, st);
-    launch_attention_simt<WT>(ctx->q, pk, pv, ctx->ks, ctx->vs, ctx->o, T, S, P, k.max_prefix_len, k.n_q_heads,
-                              k.n_kv_heads, D, prefix_batch_stride, k.suffix_mask, st);
-    launch_linear<WT>(ctx->o, Q, (const WT*)L.o, nullptr, ctx->h, w, T, w, Q, EPI_ADD, st);
-    launch_rmsnorm(ctx->h, L.g_mlp, ctx->u, T, w, k.rms_eps, st);
-    launch_linear<WT>(ctx->u, w, (const WT*)L.gu, nullptr, ctx->gu, 2 * F, T, 2 * F, w, EPI_STORE, st);
-    launch_geglu(ctx->gu, ctx->m, T, F, st);
-    launch_linear<WT>(ctx->m, F, (const WT*)L.down, nullptr, ctx->h, w, T, w, F, EPI_ADD, st);
-  }
+                   ctx->W.ai_b, c, c_stride, ctx->h, G, k.width, ctx->S, k.action_dim, k.state_dim, st);
+  simt_layers<WT>(ctx, G, P, prefix_batch_stride, rope_cs, rope_sn, st);
 }
 
 // c(t) = time_mlp_out(swish(time_mlp_in(e(t)))) for n times (taus or the Euler schedule).
@@ -229,18 +244,141 @@ rtv_status get_graph(rtv_ctx* ctx, int kind, int n, int batch, GraphEntry** out)
   return RTV_OK;
 }
 
-// Name -> (expected shape, destination) table for rtv_load_expert.
-struct Slot {
-  std::vector<long long> shape;
-  int dtype;          // expected input dtype
-  void** dst_ptr;     // destination pointer (allocated on load)
-  size_t dst_offset;  // byte offset inside a packed destination (qkv / gu), or 0
-  void** pack_base;   // packed destination base (qkv/gu) or nullptr
-  size_t pack_bytes;  // total bytes of the packed destination
-  bool seen = false;
-};
-
 }  // namespace
+
+namespace rtv {
+
+rtv_status ctx_create(const rtv_expert_config& k, int cuda_device, int S, bool block_only, rtv_ctx** out) {
+  *out = nullptr;
+  rtv_ctx* ctx = new rtv_ctx();
+  ctx->cfg = k;
+  ctx->device = cuda_device;
+  ctx->block_only = block_only;
+  DeviceGuard dg(cuda_device);
+  ctx->S = S;
+  ctx->H = S - 1;
+  ctx->Q = k.n_q_heads * k.head_dim;
+  ctx->KV = k.n_kv_heads * k.head_dim;
+  ctx->Gmax = k.max_batch > k.max_taus ? k.max_batch : k.max_taus;
+  ctx->Tmax = ctx->Gmax * ctx->S;
+  ctx->elt = (int)dtype_size(k.dtype);
+  const int w = k.width, F = k.mlp_dim, D = k.head_dim;
+  const size_t T = ctx->Tmax;
+  const int H = ctx->H > 0 ? ctx->H : 1;
+  rtv_status s = RTV_OK;
+  auto A = [&](float** p, size_t n) { if (s == RTV_OK) s = dev_alloc_t(ctx, p, n); };
+  A(&ctx->h, T * w);
+  A(&ctx->u, T * w);
+  A(&ctx->qkv, T * (ctx->Q + 2 * ctx->KV));
+  A(&ctx->q, T * ctx->Q);
+  A(&ctx->o, T * ctx->Q);
+  A(&ctx->gu, T * 2 * F);
+  A(&ctx->m, T * F);
+  A(&ctx->ks, (size_t)ctx->Gmax * ctx->KV * ctx->S);
+  A(&ctx->vs, (size_t)ctx->Gmax * ctx->KV * ctx->S);
+  A(&ctx->x, (size_t)ctx->Gmax * H * k.action_dim);
+  A(&ctx->v, (size_t)ctx->Gmax * H * k.action_dim);
+  A(&ctx->state, (size_t)ctx->Gmax * k.state_dim);
+  const size_t rows_e = T > 64 ? T : 64;   // e/z scratch rows (>= the Euler schedule length limit)
+  A(&ctx->e_tmp, rows_e * w);
+  A(&ctx->z_tmp, rows_e * w);
+  A(&ctx->c_verify, (size_t)(ctx->Gmax) * w);
+  A(&ctx->draft, (size_t)H * k.action_dim);
+  A(&ctx->eps, (size_t)H * k.action_dim);
+  A(&ctx->taus, (size_t)(ctx->Gmax > 0 ? ctx->Gmax : 1));
+  A(&ctx->vparams, 4);
+  A(&ctx->dist, (size_t)(ctx->Gmax > 0 ? ctx->Gmax : 1) * H);
+  if (s == RTV_OK) s = dev_alloc_t(ctx, &ctx->accepted, 1);
+  if (s == RTV_OK) s = dev_alloc_t(ctx, &ctx->flags, 1);
+  if (s == RTV_OK) s = dev_alloc_t(ctx, &ctx->status, 1);
+  void* kvp = nullptr;
+  if (s == RTV_OK)
+    s = dev_alloc(ctx, &kvp, (size_t)k.n_layers * 2 * k.max_batch * k.n_kv_heads * k.max_prefix_len * D * ctx->elt);
+  ctx->prefix_kv = kvp;
+  if (s == RTV_OK && cudaMemset(ctx->status, 0, sizeof(unsigned)) != cudaSuccess) s = RTV_ERR_CUDA;
+  if (s == RTV_OK && cudaStreamCreateWithFlags(&ctx->cap_stream, cudaStreamNonBlocking) != cudaSuccess)
+    s = RTV_ERR_CUDA;
+  if (s == RTV_OK && k.dtype == RTV_BF16) {
+    const char* env = getenv("RTV_PATH");
+    const bool want_simt = env && strcmp(env, "simt") == 0;
+    if (!want_simt) s = fast_create(ctx);
+  }
+  if (s == RTV_OK && k.mlp_dtype == RTV_FP8_E4M3 && !ctx->use_fast) s = RTV_ERR_UNSUPPORTED;   // no SIMT FP8
+  if (s != RTV_OK) {
+    rtv_destroy(ctx);
+    return s;
+  }
+  *out = ctx;
+  return RTV_OK;
+}
+
+void add_layer_slots(rtv_ctx* ctx, SlotTable& slots, const std::string& p, LayerW& L) {
+  const rtv_expert_config& k = ctx->cfg;
+  const long long w = k.width, F = k.mlp_dim, Q = ctx->Q, KV = ctx->KV;
+  const int md = k.dtype;
+  const size_t e = ctx->elt;
+  slots[p + "attn_norm.g"] = ParamSlot{{w}, RTV_F32, (void**)&L.g_attn, 0, nullptr, 0};
+  slots[p + "mlp_norm.g"] = ParamSlot{{w}, RTV_F32, (void**)&L.g_mlp, 0, nullptr, 0};
+  const size_t qkv_bytes = (size_t)(Q + 2 * KV) * w * e;
+  slots[p + "q_proj.w"] = ParamSlot{{Q, w}, md, nullptr, 0, &L.qkv, qkv_bytes};
+  slots[p + "k_proj.w"] = ParamSlot{{KV, w}, md, nullptr, (size_t)Q * w * e, &L.qkv, qkv_bytes};
+  slots[p + "v_proj.w"] = ParamSlot{{KV, w}, md, nullptr, (size_t)(Q + KV) * w * e, &L.qkv, qkv_bytes};
+  slots[p + "o_proj.w"] = ParamSlot{{w, Q}, md, &L.o, 0, nullptr, 0};
+  const int mdt = k.mlp_dtype;
+  const size_t em = dtype_size(mdt);
+  const size_t gu_bytes = (size_t)2 * F * w * em;
+  slots[p + "gate_proj.w"] = ParamSlot{{F, w}, mdt, nullptr, 0, &L.gu, gu_bytes};
+  slots[p + "up_proj.w"] = ParamSlot{{F, w}, mdt, nullptr, (size_t)F * w * em, &L.gu, gu_bytes};
+  slots[p + "down_proj.w"] = ParamSlot{{w, F}, mdt, &L.down, 0, nullptr, 0};
+  if (mdt == RTV_FP8_E4M3) {
+    slots[p + "gate_proj.s"] = ParamSlot{{F}, RTV_F32, nullptr, 0, (void**)&L.gu_s, (size_t)2 * F * 4};
+    slots[p + "up_proj.s"] = ParamSlot{{F}, RTV_F32, nullptr, (size_t)F * 4, (void**)&L.gu_s, (size_t)2 * F * 4};
+    slots[p + "down_proj.s"] = ParamSlot{{w}, RTV_F32, (void**)&L.down_s, 0, nullptr, 0};
+  }
+}
+
+rtv_status load_slots(rtv_ctx* ctx, SlotTable& slots, const rtv_tensor* params, int n_params) {
+  // validate every entry first: nothing is allocated on a bad table
+  for (int i = 0; i < n_params; ++i) {
+    const rtv_tensor& t = params[i];
+    if (!t.name || !t.data) return fail(ctx, RTV_ERR_ARG, "parameter with null name or data");
+    auto it = slots.find(t.name);
+    if (it == slots.end()) return fail(ctx, RTV_ERR_ARG, std::string("unknown parameter ") + t.name);
+    ParamSlot& sl = it->second;
+    if (sl.seen) return fail(ctx, RTV_ERR_ARG, std::string("duplicate parameter ") + t.name);
+    if (t.dtype != sl.dtype) return fail(ctx, RTV_ERR_ARG, std::string("wrong dtype for ") + t.name);
+    if (t.ndim != (int)sl.shape.size()) return fail(ctx, RTV_ERR_SHAPE, std::string("wrong rank for ") + t.name);
+    for (int d = 0; d < t.ndim; ++d)
+      if (t.shape[d] != sl.shape[d]) return fail(ctx, RTV_ERR_SHAPE, std::string("wrong shape for ") + t.name);
+    sl.seen = true;
+  }
+  for (auto& kv : slots)
+    if (!kv.second.seen) {
+      for (auto& kv2 : slots) kv2.second.seen = false;
+      return fail(ctx, RTV_ERR_ARG, "missing parameter " + kv.first);
+    }
+
+  // allocate and copy
+  for (int i = 0; i < n_params; ++i) {
+    const rtv_tensor& t = params[i];
+    ParamSlot& sl = slots[t.name];
+    size_t n = 1;
+    for (long long d : sl.shape) n *= (size_t)d;
+    const size_t bytes = n * dtype_size(sl.dtype);
+    void* dst = nullptr;
+    if (sl.pack_base) {
+      if (!*sl.pack_base) TRY(dev_alloc(ctx, sl.pack_base, sl.pack_bytes));
+      dst = (char*)*sl.pack_base + sl.dst_offset;
+    } else {
+      TRY(dev_alloc(ctx, sl.dst_ptr, bytes));
+      dst = *sl.dst_ptr;
+    }
+    CK(cudaMemcpy(dst, t.data, bytes, cudaMemcpyDefault));
+  }
+  return RTV_OK;
+}
+
+}  // namespace rtv
 
 // ===========================================================================
 // C ABI
@@ -270,84 +408,27 @@ rtv_status rtv_create(const rtv_expert_config* cfg_in, int cuda_device, rtv_ctx*
     cudaGetLastError();
     return RTV_ERR_CUDA;
   }
-  rtv_ctx* ctx = new rtv_ctx();
-  ctx->cfg = k;
-  ctx->device = cuda_device;
-  DeviceGuard dg(cuda_device);
-  ctx->S = 1 + k.chunk_len;
-  ctx->H = k.chunk_len;
-  ctx->Q = k.n_q_heads * k.head_dim;
-  ctx->KV = k.n_kv_heads * k.head_dim;
-  ctx->Gmax = k.max_batch > k.max_taus ? k.max_batch : k.max_taus;
-  ctx->Tmax = ctx->Gmax * ctx->S;
-  ctx->elt = (int)dtype_size(k.dtype);
-  const int w = k.width, F = k.mlp_dim, D = k.head_dim;
-  const size_t T = ctx->Tmax;
-  rtv_status s = RTV_OK;
-  auto A = [&](float** p, size_t n) { if (s == RTV_OK) s = dev_alloc_t(ctx, p, n); };
-  A(&ctx->h, T * w);
-  A(&ctx->u, T * w);
-  A(&ctx->qkv, T * (ctx->Q + 2 * ctx->KV));
-  A(&ctx->q, T * ctx->Q);
-  A(&ctx->o, T * ctx->Q);
-  A(&ctx->gu, T * 2 * F);
-  A(&ctx->m, T * F);
-  A(&ctx->ks, (size_t)ctx->Gmax * ctx->KV * ctx->S);
-  A(&ctx->vs, (size_t)ctx->Gmax * ctx->KV * ctx->S);
-  A(&ctx->x, (size_t)ctx->Gmax * ctx->H * k.action_dim);
-  A(&ctx->v, (size_t)ctx->Gmax * ctx->H * k.action_dim);
-  A(&ctx->state, (size_t)ctx->Gmax * k.state_dim);
-  const size_t rows_e = T > 64 ? T : 64;   // e/z scratch rows (>= the Euler schedule length limit)
-  A(&ctx->e_tmp, rows_e * w);
-  A(&ctx->z_tmp, rows_e * w);
-  A(&ctx->c_verify, (size_t)(ctx->Gmax) * w);
-  A(&ctx->draft, (size_t)ctx->H * k.action_dim);
-  A(&ctx->eps, (size_t)ctx->H * k.action_dim);
-  A(&ctx->taus, (size_t)(ctx->Gmax > 0 ? ctx->Gmax : 1));
-  A(&ctx->vparams, 4);
-  A(&ctx->dist, (size_t)(ctx->Gmax > 0 ? ctx->Gmax : 1) * ctx->H);
-  if (s == RTV_OK) s = dev_alloc_t(ctx, &ctx->accepted, 1);
-  if (s == RTV_OK) s = dev_alloc_t(ctx, &ctx->flags, 1);
-  if (s == RTV_OK) s = dev_alloc_t(ctx, &ctx->status, 1);
-  void* kvp = nullptr;
-  if (s == RTV_OK)
-    s = dev_alloc(ctx, &kvp, (size_t)k.n_layers * 2 * k.max_batch * k.n_kv_heads * k.max_prefix_len * D * ctx->elt);
-  ctx->prefix_kv = kvp;
-  if (s == RTV_OK && cudaMemset(ctx->status, 0, sizeof(unsigned)) != cudaSuccess) s = RTV_ERR_CUDA;
-  if (s == RTV_OK && cudaStreamCreateWithFlags(&ctx->cap_stream, cudaStreamNonBlocking) != cudaSuccess)
-    s = RTV_ERR_CUDA;
-  if (s == RTV_OK && k.dtype == RTV_BF16) {
-    const char* env = getenv("RTV_PATH");
-    const bool want_simt = env && strcmp(env, "simt") == 0;
-    if (!want_simt) s = fast_create(ctx);
-  }
-  if (s == RTV_OK && k.mlp_dtype == RTV_FP8_E4M3 && !ctx->use_fast) s = RTV_ERR_UNSUPPORTED;   // no SIMT FP8
-  if (s != RTV_OK) {
-    rtv_destroy(ctx);
-    return s;
-  }
-  *out = ctx;
-  return RTV_OK;
+  return ctx_create(k, cuda_device, 1 + k.chunk_len, false, out);
 }
 
 rtv_status rtv_load_expert(rtv_ctx* ctx, const rtv_tensor* params, int n_params) {
   if (!ctx) return RTV_ERR_ARG;
   if (!params || n_params <= 0) return fail(ctx, RTV_ERR_ARG, "no parameters");
   if (ctx->loaded) return fail(ctx, RTV_ERR_STATE, "expert already loaded");
+  if (ctx->block_only) return fail(ctx, RTV_ERR_STATE, "not an expert context");
   DeviceGuard dg(ctx->device);
   const rtv_expert_config& k = ctx->cfg;
-  const long long w = k.width, A = k.action_dim, Sd = k.state_dim, F = k.mlp_dim, Q = ctx->Q, KV = ctx->KV;
+  const long long w = k.width, A = k.action_dim, Sd = k.state_dim;
   const int md = k.dtype;
-  const size_t e = ctx->elt;
   ExpertW& W = ctx->W;
   W.layers.assign(k.n_layers, LayerW());
 
-  std::unordered_map<std::string, Slot> slots;
+  SlotTable slots;
   auto mat = [&](const std::string& n, long long r, long long c, void** dst) {
-    slots[n] = Slot{{r, c}, md, dst, 0, nullptr, 0};
+    slots[n] = ParamSlot{{r, c}, md, dst, 0, nullptr, 0};
   };
   auto vec = [&](const std::string& n, long long r, float** dst) {
-    slots[n] = Slot{{r}, RTV_F32, (void**)dst, 0, nullptr, 0};
+    slots[n] = ParamSlot{{r}, RTV_F32, (void**)dst, 0, nullptr, 0};
   };
   mat("state_proj.w", w, Sd, &W.sp_w);
   vec("state_proj.b", w, &W.sp_b);
@@ -360,66 +441,9 @@ rtv_status rtv_load_expert(rtv_ctx* ctx, const rtv_tensor* params, int n_params)
   vec("final_norm.g", w, &W.g_final);
   mat("action_out_proj.w", A, w, &W.ao_w);
   vec("action_out_proj.b", A, &W.ao_b);
-  for (int l = 0; l < k.n_layers; ++l) {
-    const std::string p = "layers." + std::to_string(l) + ".";
-    LayerW& L = W.layers[l];
-    vec(p + "attn_norm.g", w, &L.g_attn);
-    vec(p + "mlp_norm.g", w, &L.g_mlp);
-    const size_t qkv_bytes = (size_t)(Q + 2 * KV) * w * e;
-    slots[p + "q_proj.w"] = Slot{{Q, w}, md, nullptr, 0, &L.qkv, qkv_bytes};
-    slots[p + "k_proj.w"] = Slot{{KV, w}, md, nullptr, (size_t)Q * w * e, &L.qkv, qkv_bytes};
-    slots[p + "v_proj.w"] = Slot{{KV, w}, md, nullptr, (size_t)(Q + KV) * w * e, &L.qkv, qkv_bytes};
-    mat(p + "o_proj.w", w, Q, &L.o);
-    const int mdt = k.mlp_dtype;
-    const size_t em = dtype_size(mdt);
-    const size_t gu_bytes = (size_t)2 * F * w * em;
-    slots[p + "gate_proj.w"] = Slot{{F, w}, mdt, nullptr, 0, &L.gu, gu_bytes};
-    slots[p + "up_proj.w"] = Slot{{F, w}, mdt, nullptr, (size_t)F * w * em, &L.gu, gu_bytes};
-    slots[p + "down_proj.w"] = Slot{{w, F}, mdt, &L.down, 0, nullptr, 0};
-    if (mdt == RTV_FP8_E4M3) {
-      slots[p + "gate_proj.s"] = Slot{{F}, RTV_F32, nullptr, 0, (void**)&L.gu_s, (size_t)2 * F * 4};
-      slots[p + "up_proj.s"] = Slot{{F}, RTV_F32, nullptr, (size_t)F * 4, (void**)&L.gu_s, (size_t)2 * F * 4};
-      vec(p + "down_proj.s", w, &L.down_s);
-    }
-  }
-
-  // validate every entry first: nothing is allocated on a bad table
-  for (int i = 0; i < n_params; ++i) {
-    const rtv_tensor& t = params[i];
-    if (!t.name || !t.data) return fail(ctx, RTV_ERR_ARG, "parameter with null name or data");
-    auto it = slots.find(t.name);
-    if (it == slots.end()) return fail(ctx, RTV_ERR_ARG, std::string("unknown parameter ") + t.name);
-    Slot& sl = it->second;
-    if (sl.seen) return fail(ctx, RTV_ERR_ARG, std::string("duplicate parameter ") + t.name);
-    if (t.dtype != sl.dtype) return fail(ctx, RTV_ERR_ARG, std::string("wrong dtype for ") + t.name);
-    if (t.ndim != (int)sl.shape.size()) return fail(ctx, RTV_ERR_SHAPE, std::string("wrong rank for ") + t.name);
-    for (int d = 0; d < t.ndim; ++d)
-      if (t.shape[d] != sl.shape[d]) return fail(ctx, RTV_ERR_SHAPE, std::string("wrong shape for ") + t.name);
-    sl.seen = true;
-  }
-  for (auto& kv : slots)
-    if (!kv.second.seen) {
-      for (auto& kv2 : slots) kv2.second.seen = false;
-      return fail(ctx, RTV_ERR_ARG, "missing parameter " + kv.first);
-    }
-
-  // allocate and copy
-  for (int i = 0; i < n_params; ++i) {
-    const rtv_tensor& t = params[i];
-    Slot& sl = slots[t.name];
-    size_t n = 1;
-    for (long long d : sl.shape) n *= (size_t)d;
-    const size_t bytes = n * dtype_size(sl.dtype);
-    void* dst = nullptr;
-    if (sl.pack_base) {
-      if (!*sl.pack_base) TRY(dev_alloc(ctx, sl.pack_base, sl.pack_bytes));
-      dst = (char*)*sl.pack_base + sl.dst_offset;
-    } else {
-      TRY(dev_alloc(ctx, sl.dst_ptr, bytes));
-      dst = *sl.dst_ptr;
-    }
-    CK(cudaMemcpy(dst, t.data, bytes, cudaMemcpyDefault));
-  }
+  for (int l = 0; l < k.n_layers; ++l)
+    add_layer_slots(ctx, slots, "layers." + std::to_string(l) + ".", W.layers[l]);
+  TRY(load_slots(ctx, slots, params, n_params));
   if (ctx->use_fast) TRY(fast_load(ctx, params, n_params));
   CK(cudaDeviceSynchronize());
   ctx->loaded = true;

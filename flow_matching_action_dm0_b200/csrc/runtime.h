@@ -7,6 +7,7 @@
 #include <map>
 #include <string>
 #include <tuple>
+#include <unordered_map>
 #include <vector>
 
 #include "../../include/rtv.h"
@@ -44,6 +45,19 @@ struct GraphEntry {
 
 struct FastPath;  // tensor-core path state (kernels_tc.cu)
 
+// One named parameter of a load table: expected shape and dtype, and where it
+// goes (its own allocation, or an offset inside a packed allocation).
+struct ParamSlot {
+  std::vector<long long> shape;
+  int dtype;          // expected input dtype
+  void** dst_ptr;     // destination pointer (allocated on load)
+  size_t dst_offset;  // byte offset inside a packed destination (qkv / gu), or 0
+  void** pack_base;   // packed destination base (qkv/gu) or nullptr
+  size_t pack_bytes;  // total bytes of the packed destination
+  bool seen = false;
+};
+using SlotTable = std::unordered_map<std::string, ParamSlot>;
+
 }  // namespace rtv
 
 struct rtv_ctx {
@@ -54,6 +68,9 @@ struct rtv_ctx {
   int prefix_len = 0, prefix_batch = 0;
   bool have_prefix = false;
   bool use_fast = false;   // tcgen05 path
+  // A bare stack of layers (the FLASH draft model's block): no suffix
+  // embedding, time condition or output head of its own.
+  bool block_only = false;
 
   // derived sizes
   int S = 0, H = 0, Q = 0, KV = 0, Gmax = 0, Tmax = 0, elt = 4;
@@ -77,3 +94,20 @@ struct rtv_ctx {
 
   rtv::FastPath* fast = nullptr;
 };
+
+namespace rtv {
+
+// Allocate a context's static buffers for suffixes of S token rows and pick
+// its kernel path.  The caller has validated cfg and the device.
+rtv_status ctx_create(const rtv_expert_config& cfg, int cuda_device, int S, bool block_only, rtv_ctx** out);
+// Entries of one layer's parameters under the name prefix p.
+void add_layer_slots(rtv_ctx* ctx, SlotTable& slots, const std::string& p, LayerW& L);
+// Validate a parameter list against the table (every name exactly once,
+// dtype and shape), then allocate and copy.  Nothing is allocated on a bad list.
+rtv_status load_slots(rtv_ctx* ctx, SlotTable& slots, const rtv_tensor* params, int n_params);
+// The SIMT layers over G suffixes of ctx->S rows (residual stream ctx->h).
+template <typename WT>
+void simt_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, const float* rope_cs, const float* rope_sn,
+                 cudaStream_t st);
+
+}  // namespace rtv

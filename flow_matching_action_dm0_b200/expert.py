@@ -66,6 +66,55 @@ def _stream(stream) -> int:
     return int(getattr(stream, "cuda_stream", stream))
 
 
+def _dtype_code(name: str, a, matrix_dtype: int, overrides) -> int:
+    if overrides and name in overrides:
+        return overrides[name]
+    if hasattr(a, "dtype") and str(a.dtype) in ("torch.bfloat16",):
+        return L.RTV_BF16
+    if hasattr(a, "dtype") and str(a.dtype) in ("torch.float8_e4m3fn",):
+        return L.RTV_FP8_E4M3
+    if isinstance(a, np.ndarray) and a.dtype == np.uint16:
+        return L.RTV_BF16
+    if isinstance(a, np.ndarray) and a.dtype == np.uint8:
+        return L.RTV_FP8_E4M3
+    return matrix_dtype if len(a.shape) == 2 else L.RTV_F32
+
+
+def to_dtype_bits(a, dtype_code: int, what: str):
+    """numpy float32 values given in bf16 -> their uint16 bits (checked)."""
+    if isinstance(a, np.ndarray) and dtype_code == L.RTV_BF16 and a.dtype == np.float32:
+        bits = np.ascontiguousarray(a).view(np.uint32)
+        if np.any(bits & np.uint32(0xFFFF)):
+            raise ValueError(f"{what}: float32 values are not bf16-representable")
+        return (bits >> np.uint32(16)).astype(np.uint16)
+    return a
+
+
+def make_tensors(weights: Dict[str, object], matrix_dtype: int, overrides: Optional[Dict[str, int]] = None):
+    """rtv_tensor entries for a name -> array table, and the arrays they point
+    into (keep them alive during the load call).  2-D arrays are given in
+    matrix_dtype unless their own dtype or ``overrides`` says otherwise;
+    float32 numpy values of a bf16 matrix are passed as their bf16 bits."""
+    tensors, keep = [], []
+    for name, a in weights.items():
+        code = _dtype_code(name, a, matrix_dtype, overrides)
+        a = to_dtype_bits(a, code, name)
+        if isinstance(a, np.ndarray):
+            a = np.ascontiguousarray(a)
+        ptr, dev = _ptr(a)
+        keep.append(a)
+        t = L.rtv_tensor()
+        t.name = name.encode()
+        t.data = ptr
+        t.dtype = code
+        t.ndim = len(a.shape)
+        for i, d in enumerate(a.shape):
+            t.shape[i] = int(d)
+        t.is_device = int(dev)
+        tensors.append(t)
+    return tensors, keep
+
+
 class ActionExpert:
     def __init__(self, shape, device: int = 0, max_batch: Optional[int] = None, max_taus: int = 4,
                  max_prefix_len: Optional[int] = None):
@@ -79,53 +128,15 @@ class ActionExpert:
     def load(self, weights: Dict[str, object], mlp_dtype_codes: Optional[Dict[str, int]] = None):
         """weights: name -> array.  float32 numpy arrays are accepted for bf16
         matrices when their values are bf16-representable (passed as bits)."""
-        tensors, keep = [], []
-        for name, a in weights.items():
-            code = self._code_for(name, a, mlp_dtype_codes)
-            if isinstance(a, np.ndarray) and code == L.RTV_BF16 and a.dtype == np.float32:
-                bits = np.ascontiguousarray(a).view(np.uint32)
-                if np.any(bits & np.uint32(0xFFFF)):
-                    raise ValueError(f"{name}: float32 values are not bf16-representable")
-                a = (bits >> np.uint32(16)).astype(np.uint16)
-            if isinstance(a, np.ndarray):
-                a = np.ascontiguousarray(a)
-            ptr, dev = _ptr(a)
-            keep.append(a)
-            t = L.rtv_tensor()
-            t.name = name.encode()
-            t.data = ptr
-            t.dtype = code
-            t.ndim = len(a.shape)
-            for i, d in enumerate(a.shape):
-                t.shape[i] = int(d)
-            t.is_device = int(dev)
-            tensors.append(t)
+        tensors, keep = make_tensors(weights, self.cfg.dtype, mlp_dtype_codes)
         L.rtv_load_expert(self.h, tensors)
         del keep
-
-    def _code_for(self, name: str, a, overrides) -> int:
-        if overrides and name in overrides:
-            return overrides[name]
-        if hasattr(a, "dtype") and str(a.dtype) in ("torch.bfloat16",):
-            return L.RTV_BF16
-        if hasattr(a, "dtype") and str(a.dtype) in ("torch.float8_e4m3fn",):
-            return L.RTV_FP8_E4M3
-        if isinstance(a, np.ndarray) and a.dtype == np.uint16:
-            return L.RTV_BF16
-        if isinstance(a, np.ndarray) and a.dtype == np.uint8:
-            return L.RTV_FP8_E4M3
-        ndim = len(a.shape)
-        return self.cfg.dtype if ndim == 2 else L.RTV_F32
 
     # ------------------------------------------------------------------
     def set_prefix_kv(self, kv, prefix_len: Optional[int] = None, batch: Optional[int] = None, stream=None):
         """kv [L][2][B][P][Hkv][D] in the config dtype (torch tensor, or numpy
         float32 / uint16 bf16 bits)."""
-        if isinstance(kv, np.ndarray) and self.cfg.dtype == L.RTV_BF16 and kv.dtype == np.float32:
-            bits = np.ascontiguousarray(kv).view(np.uint32)
-            if np.any(bits & np.uint32(0xFFFF)):
-                raise ValueError("prefix kv float32 values are not bf16-representable")
-            kv = (bits >> np.uint32(16)).astype(np.uint16)
+        kv = to_dtype_bits(kv, self.cfg.dtype, "prefix kv")
         b = int(batch if batch is not None else kv.shape[2])
         p = int(prefix_len if prefix_len is not None else kv.shape[3])
         ptr, _ = _ptr(kv)

@@ -13,9 +13,11 @@
  *           startup graph capture with static addresses, one replay, step
  *           count fixed at capture.
  *   [FLASH] "Realtime-VLA FLASH" sec. 02 (interpolate, predict, rebuild the
- *           endpoint, compare), sec. 03.2 (accept the prefix below delta at
- *           every verification time; zero length -> full path), sec. 03.3
- *           (gripper switch -> full path).
+ *           endpoint, compare), sec. 03.1 (draft model: one Gemma block and
+ *           a linear action head over learnable action queries and the
+ *           current image features, about 110M parameters), sec. 03.2
+ *           (accept the prefix below delta at every verification time; zero
+ *           length -> full path), sec. 03.3 (gripper switch -> full path).
  *
  * Conventions shared by every call:
  *   - Matrices are row-major [out][in].  Activations and actions are fp32.
@@ -207,6 +209,89 @@ int rtv_graph_kernel_count(rtv_ctx* ctx, int n, int is_verify);
 
 /* Release every resource of the context.  NULL is accepted. */
 void rtv_destroy(rtv_ctx* ctx);
+
+
+/* ------------------------------------------------------------------------
+ * FLASH draft model ([FLASH] 03.1) and dual-path round ([FLASH] 03).
+ *
+ * The draft model is one Gemma block and a linear action head.  The image
+ * features of one observation (n_vis tokens of `width`) are followed by
+ * n_queries learnable action queries; the block (RMSNorm with gain 1+g,
+ * q/k/v projections, RoPE at positions 0..n_vis+n_queries-1, softmax
+ * attention in which every row sees every row, o_proj + residual, RMSNorm,
+ * GeGLU MLP + residual) runs once, and the head maps each query row to one
+ * action: chunk[h] = action_head.w . x[n_vis + h] + action_head.b.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  int width, n_q_heads, n_kv_heads, head_dim, mlp_dim;
+  int n_queries;      /* H: action queries = rows of the candidate chunk (1..64)  */
+  int action_dim;     /* A                                                        */
+  int max_vis;        /* largest n_vis a call may pass                            */
+  int max_batch;      /* largest batch a call may pass                            */
+  int dtype;          /* RTV_F32 | RTV_BF16: weight matrices and image features   */
+  float rms_eps;
+  float rope_theta;   /* 0 disables rotary embedding                              */
+  long long barrier_timeout_ns;   /* 0 = library default (100 ms)                 */
+} rtv_draft_config;
+
+typedef struct rtv_draft rtv_draft;
+
+/* Create a draft model on CUDA device `cuda_device`; allocates its static
+ * buffers for the maxima.  width must be a multiple of 128.  *out is NULL on
+ * failure.  Returns RTV_ERR_ARG on a bad config, RTV_ERR_CUDA on a bad
+ * device, RTV_ERR_OOM when the buffers do not fit. */
+rtv_status rtv_draft_create(const rtv_draft_config* cfg, int cuda_device, rtv_draft** out);
+
+/* Copy and pack the draft parameters (rtv_tensor as for rtv_load_expert;
+ * w = width, F = mlp_dim, Q = n_q_heads*head_dim, KV = n_kv_heads*head_dim,
+ * H = n_queries, A = action_dim):
+ *   action_queries [H][w] (RTV_F32)
+ *   attn_norm.g [w]  q_proj.w [Q][w]  k_proj.w [KV][w]  v_proj.w [KV][w]
+ *   o_proj.w [w][Q]  mlp_norm.g [w]  gate_proj.w [F][w]  up_proj.w [F][w]
+ *   down_proj.w [w][F]  action_head.w [A][w]  action_head.b [A]
+ * Matrices in the config dtype, vectors in RTV_F32; every name exactly once.
+ * Synchronous. */
+rtv_status rtv_draft_load(rtv_draft* d, const rtv_tensor* params, int n_params);
+
+/* Candidate chunks chunk_out [batch][H][A] (fp32) from the image features
+ * vis [batch][n_vis][width] (config dtype), each batch element on its own.
+ * vis and chunk_out may be device or host memory (host copies are enqueued
+ * on `stream`).  n_vis <= max_vis, batch <= max_batch.  Asynchronous; the
+ * first call for a given (n_vis, batch) captures a CUDA graph (not on
+ * `stream`), later calls replay it. */
+rtv_status rtv_draft_forward(rtv_draft* d, const void* vis, int n_vis, int batch, float* chunk_out,
+                             rtv_stream stream);
+
+/* One FLASH round for one observation ([FLASH] 03): draft the chunk from
+ * vis [n_vis][width], verify it with the expert `ctx` (as rtv_verify, with
+ * noise [H][A], state [Sd], taus, delta, gripper_dim), and when the verdict
+ * is a fallback (accepted length 0 or a gripper switch) run the full path,
+ * rtv_denoise(ctx, noise, state, n_steps), from the same noise.  Writes the
+ * chunk [H][A] to actions_out (the draft, or the denoised chunk), and to
+ * host memory *accepted_len, *flags (RTV_FLAG_*) and *used_full (1 = the
+ * full path ran).  The expert's prefix KV must be installed with batch 1;
+ * its chunk_len and action_dim must equal the draft's n_queries and
+ * action_dim.  Synchronous: returns once actions_out holds the chunk. */
+rtv_status rtv_flash_round(rtv_ctx* ctx, rtv_draft* d, const void* vis, int n_vis, const float* noise,
+                           const float* state, const float* taus, int n_taus, float delta, int gripper_dim,
+                           int n_steps, float* actions_out, int* accepted_len, unsigned* flags, int* used_full,
+                           rtv_stream stream);
+
+/* As rtv_device_status, for the draft model's kernels. */
+rtv_status rtv_draft_device_status(rtv_draft* d, unsigned* bits);
+
+/* Last error message of the draft model (never NULL). */
+const char* rtv_draft_last_error(rtv_draft* d);
+
+/* Kernel path of the draft model ("tcgen05", "simt"). */
+const char* rtv_draft_path_name(rtv_draft* d);
+
+/* Kernel launches of one rtv_draft_forward(n_vis, batch); -1 before its
+ * graph has been captured. */
+int rtv_draft_kernel_count(rtv_draft* d, int n_vis, int batch);
+
+/* Release every resource of the draft model.  NULL is accepted. */
+void rtv_draft_destroy(rtv_draft* d);
 
 #ifdef __cplusplus
 }

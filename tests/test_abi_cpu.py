@@ -60,3 +60,30 @@ def test_create_without_gpu_reports_cuda_error():
     h = C.c_void_p()
     assert L.load_library().rtv_create(C.byref(cfg), 0, C.byref(h)) == L.RTV_ERR_CUDA
     assert not h.value
+
+
+def test_draft_null_arguments_are_refused():
+    lib = L.load_library()
+    assert lib.rtv_draft_create(None, 0, None) == L.RTV_ERR_ARG
+    d = C.c_void_p()
+    assert lib.rtv_draft_create(None, 0, C.byref(d)) == L.RTV_ERR_ARG
+    assert not d.value
+    assert lib.rtv_draft_load(None, None, 0) == L.RTV_ERR_ARG
+    assert lib.rtv_draft_forward(None, None, 1, 1, None, None) == L.RTV_ERR_ARG
+    assert lib.rtv_flash_round(None, None, None, 1, None, None, None, 1, C.c_float(0.05), 0, 10, None, None, None,
+                               None, None) == L.RTV_ERR_ARG
+    assert lib.rtv_draft_kernel_count(None, 1, 1) == -1
+    lib.rtv_draft_destroy(None)
+    assert lib.rtv_draft_last_error(None) == b"null draft model"
+
+
+@pytest.mark.parametrize("field,value", [("width", 200), ("n_queries", 0), ("n_queries", 65), ("n_kv_heads", 3),
+                                         ("max_vis", 0), ("dtype", 2)])
+def test_invalid_draft_config_is_refused_before_device_use(field, value):
+    from synthetic import get_draft_config
+    from flow_matching_action_dm0_b200 import make_draft_config
+    cfg = make_draft_config(get_draft_config("draft-tiny"))
+    setattr(cfg, field, value)
+    d = C.c_void_p()
+    assert L.load_library().rtv_draft_create(C.byref(cfg), 0, C.byref(d)) == L.RTV_ERR_ARG
+    assert not d.value
