@@ -5,6 +5,7 @@ expert (18 layers, width 1024, 8 q / 1 kv heads, head_dim 256, GeGLU 4096,
 bandwidth it achieves.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --workload flash-draft      # the FLASH draft model alone
 
 One "step" is one call of rtv_denoise: the whole hot path (10 Euler steps
 through the expert) over one batch of synthetic input.  With N > 1 the
@@ -37,6 +38,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "10-step action-chunk latency (us) and achieved HBM GB/s vs 8 TB/s roofline"
+DRAFT_METRIC = "FLASH draft forward latency (us): one Gemma-2B-width block + action head over 768 image tokens"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
 
@@ -186,10 +188,41 @@ def oracle_step_seconds(cfg, target_s: float, min_samples: int = 1, max_samples:
     return statistics.median(times), k
 
 
+def run_reference_draft(args, info):
+    """The CPU oracle's draft forward on the flash-draft workload: each step
+    is one whole forward (about 110M parameters x 818 rows in fp64)."""
+    from oracle import draft as OD
+    from synthetic import get_draft_config, make_draft_weights, make_visual_tokens
+    dcfg = get_draft_config(args.workload)
+    W = make_draft_weights(dcfg)
+    vis = make_visual_tokens(dcfg)[0]
+    steps = max(1, min(args.steps, 3))
+    OD.draft_forward(W, dcfg, vis)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        OD.draft_forward(W, dcfg, vis)
+    us = (time.perf_counter() - t0) / steps * 1e6
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": DRAFT_METRIC, "value": us, "unit": "us", "n_gpus": args.gpus,
+        "steps": steps, "warmup": 1, "ms_per_step": us / 1000.0, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "n_vis": dcfg.n_vis, "n_queries": dcfg.n_queries, "batch": 1},
+        "cpu_baseline": {"value": us, "unit": "us", "cores": cores, "kind": "oracle",
+                         "sample": f"{steps} whole draft forwards (fp64 numpy oracle)"},
+        "e2e": {"value": us, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(args, info):
     """The CPU oracle, as it stands, on a bounded sample of the workload:
     each step is one Euler step of the chunk, scaled to chunk latency."""
     if not info.is_main:
+        return
+    from synthetic import DRAFTS
+    if args.workload in DRAFTS:
+        run_reference_draft(args, info)
         return
     from synthetic import get_config
     cfg = get_config(args.workload, n_steps=args.n_steps)
@@ -470,6 +503,101 @@ def measure_round(ex, cfg, noise, state, stream, dev, K):
     return res
 
 
+def run_draft(args, info):
+    """The FLASH draft model alone (workload flash-draft): one step is one
+    rtv_draft_forward over one observation's 768 image tokens."""
+    import torch
+
+    from flow_matching_action_dm0_b200 import DraftModel
+    from flow_matching_action_dm0_b200 import replicas as R
+    from synthetic import f32_to_bf16_bits, get_draft_config, make_draft_weights, make_visual_tokens
+
+    dev = info.local_rank
+    torch.cuda.set_device(dev)
+    dcfg = get_draft_config(args.workload)
+    if args.batch > 0:
+        dcfg = dcfg.with_(batch=args.batch)
+    B = dcfg.batch
+    vis = make_visual_tokens(dcfg)
+    dm = DraftModel(dcfg, device=dev, max_batch=B)
+    dm.load(make_draft_weights(dcfg))
+    bits = f32_to_bf16_bits(vis).view(np.int16) if dcfg.dtype == "bf16" else vis
+    vis_t = torch.from_numpy(bits)
+    if dcfg.dtype == "bf16":
+        vis_t = vis_t.view(torch.bfloat16)
+    vis_d = vis_t.cuda(dev)
+    out_d = torch.empty((B, dcfg.n_queries, dcfg.action_dim), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    for _ in range(max(3, args.warmup)):
+        dm.forward(vis_d, out_d, stream=stream)
+    torch.cuda.synchronize(dev)
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    gpu_id = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    K = args.steps
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    R.barrier(info, dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(gpu_id) as clk:
+        start.record(stream)
+        for _ in range(K):
+            dm.forward(vis_d, out_d, stream=stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    R.barrier(info, dev)
+    ms = R.max_over_ranks(start.elapsed_time(end) / K, info, dev)
+    s, bits_ = dm.status()
+    if s != 0:
+        raise RuntimeError(f"device status {bits_:#x} after the timed region")
+    vis_h = vis_t.pin_memory()
+    out_h = torch.empty_like(out_d, device="cpu").pin_memory()
+    for _ in range(2):
+        dm.forward(vis_h, out_h, stream=stream)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        dm.forward(vis_h, out_h, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = R.max_over_ranks(e0.elapsed_time(e1) / K, info, dev)
+    kernels = dm.kernels_per_call(dcfg.n_vis, B)
+    path = dm.path
+    dm.close()
+    if not info.is_main:
+        return
+    peaks, peak_kind = load_peaks()
+    nbytes = draft_bytes(dcfg) + (B - 1) * (dcfg.n_vis * dcfg.width * 2 + dcfg.n_vis * 4 * dcfg.kv_dim)
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    peak = float(peaks["hbm_gbs"])
+    line = {
+        "metric": DRAFT_METRIC, "value": ms * 1000.0, "unit": "us", "n_gpus": info.world, "steps": K,
+        "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": dcfg.dtype, "data": "synthetic",
+        "config": {"workload": args.workload, "n_vis": dcfg.n_vis, "n_queries": dcfg.n_queries, "batch": B,
+                   "width": dcfg.width, "mlp_dim": dcfg.mlp_dim, "params": dcfg.params(),
+                   "parallelism": f"replicas x{info.world}",
+                   "l2": "inputs larger than L2: 220 MB of block weights stream from HBM every call; no flush",
+                   "path": path},
+        "roofline": {"bound": "hbm", "kernel": "whole draft graph", "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "peak_kind": f"{peak_kind} hbm_gbs",
+                     "algorithmic_bytes_per_launch": nbytes, "traffic": None},
+        "e2e": {"value": e2e_ms * 1000.0, "unit": "us", "h2d_bytes_per_step": int(vis_t.numel() * vis_t.element_size()),
+                "d2h_bytes_per_step": int(out_d.numel() * 4)},
+        "clocks": clk.summary(),
+        "gpu_launches": int(kernels * K) if kernels > 0 else None,
+    }
+    if info.world == 1 and not args.no_cpu_baseline:
+        from oracle import draft as OD
+        W = make_draft_weights(dcfg)
+        t0 = time.perf_counter()
+        OD.draft_forward(W, dcfg, vis[0])
+        per = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": per * B * 1e6, "unit": "us", "cores": blas_threads(), "kind": "oracle",
+                                "sample": "one whole draft forward of one observation (fp64 numpy oracle)"
+                                          + (f", x{B} for the batch" if B > 1 else "")}
+    print(json.dumps(line), flush=True)
+
+
 def run_trace(args):
     """One traced chunk: the library prints per-CTA phase stamps (globaltimer)
     of the projections and the attention of layer 0, first Euler step."""
@@ -499,8 +627,12 @@ def main(argv=None):
         run_reference(args, info)
         return 0
     info = R.init("nccl" if info.world > 1 else "gloo")
+    from synthetic import DRAFTS
     try:
-        run_ours(args, info)
+        if args.workload in DRAFTS:
+            run_draft(args, info)
+        else:
+            run_ours(args, info)
     finally:
         R.shutdown(info)
     return 0

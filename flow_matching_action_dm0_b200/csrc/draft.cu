@@ -101,7 +101,25 @@ rtv_status dalloc(rtv_draft* d, void** p, size_t bytes, bool zero = false) {
 // ---------------------------------------------------------------------------
 
 // Action head ([FLASH] 03.1): out[t][a] = W[a] . h[t] + b[a] for every
-// query row t.  One CTA per row, one warp per output.
+// query row t.  CTA (t, j) takes outputs 8j..8j+7 of row t, one per warp; a
+// lane reads 8 consecutive features per step (16-byte weight loads for bf16).
+__device__ __forceinline__ void load8(const float* p, float v[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float v[8]) {
+  const uint4 q = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h2[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
 template <typename WT>
 __global__ void __launch_bounds__(256) draft_head_kernel(const float* __restrict__ h, const WT* __restrict__ W,
                                                          const float* __restrict__ b, float* __restrict__ out,
@@ -109,10 +127,17 @@ __global__ void __launch_bounds__(256) draft_head_kernel(const float* __restrict
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float* hr = h + (size_t)t * w;
-  for (int a = warp; a < A; a += 8) {
+  const int a = (int)blockIdx.y * 8 + warp;
+  if (a < A) {
     const WT* wr = W + (size_t)a * w;
     float acc = 0.f;
-    for (int k = lane; k < w; k += 32) acc = fmaf(hr[k], to_f32(wr[k]), acc);
+    for (int k = lane * 8; k < w; k += 256) {   // w is a multiple of 128
+      float x[8], y[8];
+      load8(hr + k, x);
+      load8(wr + k, y);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc = fmaf(x[i], y[i], acc);
+    }
     acc = warp_sum(acc);
     if (lane == 0) out[(size_t)t * A + a] = acc + b[a];
   }
@@ -198,7 +223,8 @@ rtv_status enqueue_forward(rtv_draft* d, int V, int B, const float* cs_v, const 
     broadcast_rows_kernel<<<256, 256, 0, st>>>(d->queries, c->h, H, w, Tq);
     simt_layers<WT>(c, B, V, 1, cs_q, sn_q, st);
   }
-  draft_head_kernel<WT><<<Tq, 256, 0, st>>>(c->h, (const WT*)d->head_w, d->head_b, d->out, w, A);
+  draft_head_kernel<WT><<<dim3(Tq, (A + 7) / 8), 256, 0, st>>>(c->h, (const WT*)d->head_w, d->head_b, d->out, w,
+                                                                A);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return dfail(d, RTV_ERR_CUDA, std::string("draft launch: ") + cudaGetErrorString(e));
   return RTV_OK;

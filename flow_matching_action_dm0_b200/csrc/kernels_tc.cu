@@ -1446,6 +1446,10 @@ struct FastPath {
   // that holds tensor memory runs one CTA per SM whatever its shared memory;
   // the budget leaves room beside it for a CTA of the attention or step kernel.
   int smem_cap = 100 * 1024;
+  bool deep_single_wave = false;   // see plan_gemm (a bare block: its GEMMs have no PDL partner to leave room for)
+  // Bytes of the next projection's weights one launch brings into L2 at most
+  // (a projection larger than L2 is partly prefetched: its first bytes).
+  unsigned long long pf_cap = 48ull << 20;
   // optional phase trace of the four projections of layer 0 in the first Euler step
   unsigned long long* trace = nullptr;
   int trace_ctas[5] = {0, 0, 0, 0, 0};
@@ -1471,6 +1475,10 @@ int round_up(int x, int m) { return (x + m - 1) / m * m; }
 // go to the smaller cluster (less reduction traffic).
 GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T, bool with_in, bool f8 = false,
                    int n_tt = 1) {
+  // (With deep_single_wave, a split whose clusters are all resident at once
+  // with one CTA per SM takes the deepest ring the whole shared memory
+  // holds: more weight boxes in flight per CTA, at the price of no
+  // co-resident CTA of the next kernel.)
   GemmPlan best;
   best.n_tiles = N / 128;
   best.n_tt = n_tt;
@@ -1484,7 +1492,8 @@ GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T, bool with
     int stages = nbox;
     while (stages > 1 && total(stages) > fp->smem_cap) --stages;
     int per_sm = 2;
-    if (total(stages) > fp->smem_cap) {
+    const bool one_wave = fp->deep_single_wave && best.n_tiles * n_tt <= fp->gemm_fit_large[cs];
+    if (one_wave || total(stages) > fp->smem_cap) {
       per_sm = 1;
       stages = nbox;
       while (stages > 1 && total(stages) > kDynSmemMax) --stages;
@@ -1508,7 +1517,8 @@ GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T, bool with
 }
 
 template <int MODE>
-cudaError_t launch_gemm(const GemmArgs& a, const GemmPlan& pl, cudaStream_t st) {
+cudaError_t launch_gemm(const GemmArgs& a, const GemmPlan& pl, cudaStream_t st,
+                        unsigned long long pf_cap = ~0ull) {
   auto kern = gemm_tc_kernel<MODE>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.cs, pl.n_tiles, pl.n_tt);
@@ -1527,6 +1537,7 @@ cudaError_t launch_gemm(const GemmArgs& a, const GemmPlan& pl, cudaStream_t st) 
   GemmArgs args = a;
   args.kslice = pl.kslice;
   args.stages = pl.stages;
+  if (args.pf_bytes > pf_cap) args.pf_bytes = pf_cap;
   return cudaLaunchKernelEx(&cfg, kern, args);
 }
 
@@ -1673,6 +1684,11 @@ rtv_status fast_create(rtv_ctx* ctx) {
   }
   FastPath* fp = new FastPath();
   cudaDeviceGetAttribute(&fp->num_sms, cudaDevAttrMultiProcessorCount, dev);
+  // A bare block's GEMMs leave no room for a partner kernel: two CTAs per SM
+  // may take half of the SM's 228 KB each (less the per-CTA reservation and
+  // static shared memory), and a one-wave split the whole of it.
+  fp->deep_single_wave = ctx->block_only;
+  if (ctx->block_only) fp->smem_cap = 112 * 1024;
   // co-resident GEMM clusters by cluster size, at both shared-memory budgets
   for (int cs = 1; cs <= 16; cs <<= 1) {
     for (int big = 0; big < 2; ++big) {
@@ -1941,6 +1957,9 @@ rtv_status fast_block_prefix(rtv_ctx* ctx, const __nv_bfloat16* vis, int n_vis, 
     ctx->last_error = "no tensor-core split fits the visual-token projection";
     return RTV_ERR_UNSUPPORTED;
   }
+  if (getenv("RTV_LOG"))
+    fprintf(stderr, "[rtv] T=%d visual k/v: tiles=%d token_tiles=%d cluster=%d kslice=%d stages=%d smem=%d\n", T,
+            p.n_tiles, p.n_tt, p.cs, p.kslice, p.stages, p.smem);
   // keys and values of the visual tokens: the K and V weight tiles of the
   // layer (the q tiles are skipped), RoPE at positions 0..n_vis-1, written
   // into the cached prefix [2][Bmax][Hkv][Pmax][D] of layer 0
@@ -2123,7 +2142,7 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     a.w_tile0 = l * nq / 128;
     a.pf = (const uint8_t*)(fp->w_o + (size_t)l * w * Q);
     a.pf_bytes = (unsigned long long)w * Q * 2;
-    cudaError_t e = launch_gemm<GM_QKV>(a, p_qkv, st);
+    cudaError_t e = launch_gemm<GM_QKV>(a, p_qkv, st, fp->pf_cap);
 
     if (tc_att) {
       atc.trace = tr(l, 4);
@@ -2147,7 +2166,7 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     a.pf = fp->mlp_f8 ? fp->w_gu8 + (size_t)l * 2 * F * w : (const uint8_t*)(fp->w_gu + (size_t)l * 2 * F * w);
     a.pf_bytes = (unsigned long long)2 * F * w * (fp->mlp_f8 ? 1 : 2);
     a.g_next = Lw.g_mlp;
-    if (e == cudaSuccess) e = launch_gemm<GM_O>(a, p_o, st);
+    if (e == cudaSuccess) e = launch_gemm<GM_O>(a, p_o, st, fp->pf_cap);
 
     a = base;
     a.trace = tr(l, 2);
@@ -2159,7 +2178,7 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     a.w_tile0 = l * 2 * F / 128;
     a.pf = fp->mlp_f8 ? fp->w_down8 + (size_t)l * w * F : (const uint8_t*)(fp->w_down + (size_t)l * w * F);
     a.pf_bytes = (unsigned long long)w * F * (fp->mlp_f8 ? 1 : 2);
-    if (e == cudaSuccess) e = launch_gemm<GM_GU>(a, p_gu, st);
+    if (e == cudaSuccess) e = launch_gemm<GM_GU>(a, p_gu, st, fp->pf_cap);
 
     a = base;
     a.trace = tr(l, 3);
@@ -2172,7 +2191,7 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     a.pf = (const uint8_t*)(fp->w_qkv + (size_t)((l + 1) % k.n_layers) * nq * w);
     a.pf_bytes = (unsigned long long)nq * w * 2;
     a.g_next = (l + 1 < k.n_layers) ? ctx->W.layers[l + 1].g_attn : nullptr;
-    if (e == cudaSuccess) e = launch_gemm<GM_DOWN>(a, p_dn, st);
+    if (e == cudaSuccess) e = launch_gemm<GM_DOWN>(a, p_dn, st, fp->pf_cap);
     if (e != cudaSuccess) {
       ctx->last_error = std::string("tensor-core launch: ") + cudaGetErrorString(e);
       return RTV_ERR_CUDA;

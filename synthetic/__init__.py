@@ -7,7 +7,8 @@ attention, no time embedding, no Euler step), so the oracle and the CUDA
 path can both use it without sharing any computation.
 """
 
-from .configs import CONFIGS, DRAFTS, DraftShape, ExpertShape, get_config, get_draft_config  # noqa: F401
+from .configs import (CONFIGS, DRAFTS, PREFILLS, DraftShape, ExpertShape, PrefillShape, get_config,  # noqa: F401
+                      get_draft_config, get_prefill_config)
 from .gen import (  # noqa: F401
     bf16_bits_to_f32,
     e4m3_encode,
@@ -16,10 +17,13 @@ from .gen import (  # noqa: F401
     make_draft,
     make_draft_weights,
     make_noise,
+    make_prefill_weights,
+    make_prefix_embeddings,
     make_prefix_kv,
     make_state,
     make_visual_tokens,
     make_weights,
+    prefill_weight_names,
     round_to_bf16,
     weight_names,
 )

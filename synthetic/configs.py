@@ -25,6 +25,12 @@ current image features in one forward pass):
                  head_dim 256, GeGLU 16384: 110.1M block parameters), 50
                  queries of 32-dim actions over the 768 image tokens (3 views
                  x 256) of the pi0-bf16 observation, bf16.
+
+VLM prefill (the prefix side of the suffix loop; "DM0.5 reading guide" sec.
+5.1: the prefix is encoded once into a per-layer KV cache):
+  gemma2b-prefill  Gemma-2B-class stack: 18 layers, width 2048, 8 q / 1 kv
+                   heads, head_dim 256, GeGLU 16384, over 816 random
+                   embedding tokens, writing the pi0-bf16 expert's cache.
 """
 
 from __future__ import annotations
@@ -165,4 +171,59 @@ def get_draft_config(name: str, **overrides) -> DraftShape:
 
 def get_config(name: str, **overrides) -> ExpertShape:
     cfg = CONFIGS[name]
+    return cfg.with_(**overrides) if overrides else cfg
+
+
+@dataclass(frozen=True)
+class PrefillShape:
+    """A Gemma-style VLM stack that turns prefix embeddings into the
+    per-layer KV cache the action expert reads."""
+    name: str
+    n_layers: int
+    width: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    mlp_dim: int
+    n_tokens: int           # P, prefix tokens
+    dtype: str = "bf16"
+    rms_eps: float = 1e-6
+    rope_theta: float = 10000.0
+    weight_std: float = 0.02
+    seed: int = 0
+
+    @property
+    def q_dim(self) -> int:
+        return self.n_q_heads * self.head_dim
+
+    @property
+    def kv_dim(self) -> int:
+        return self.n_kv_heads * self.head_dim
+
+    def with_(self, **kw) -> "PrefillShape":
+        return replace(self, **kw)
+
+    def layer_params(self) -> int:
+        w, f = self.width, self.mlp_dim
+        return w * (self.q_dim + 2 * self.kv_dim) + self.q_dim * w + 3 * w * f + 2 * w
+
+    def flops(self) -> float:
+        """Dense FLOPs of the prefill: every layer but the last in full
+        (projections and attention), the last one's K/V projection only."""
+        p, w, f = self.n_tokens, self.width, self.mlp_dim
+        full = 2 * p * (w * (self.q_dim + 2 * self.kv_dim) + self.q_dim * w + 3 * w * f) + \
+            4 * p * p * self.q_dim
+        return (self.n_layers - 1) * full + 2 * p * w * 2 * self.kv_dim
+
+
+GEMMA2B_PREFILL = PrefillShape(
+    name="gemma2b-prefill", n_layers=18, width=2048, n_q_heads=8, n_kv_heads=1, head_dim=256, mlp_dim=16384,
+    n_tokens=816,
+)
+
+PREFILLS = {c.name: c for c in (GEMMA2B_PREFILL,)}
+
+
+def get_prefill_config(name: str, **overrides) -> PrefillShape:
+    cfg = PREFILLS[name]
     return cfg.with_(**overrides) if overrides else cfg

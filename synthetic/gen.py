@@ -30,7 +30,7 @@ from typing import Dict, List, Tuple
 
 import numpy as np
 
-from .configs import DraftShape, ExpertShape
+from .configs import DraftShape, ExpertShape, PrefillShape
 
 
 def _rng(seed: int, name: str) -> np.random.Generator:
@@ -241,5 +241,56 @@ def make_visual_tokens(dcfg: DraftShape, batch: int | None = None, n_vis: int | 
     v = dcfg.n_vis if n_vis is None else n_vis
     x = _normal(seed, "visual_tokens", (b, v, dcfg.width), 1.0)
     if dcfg.dtype == "bf16":
+        x = round_to_bf16(x)
+    return x
+
+
+
+# ---------------------------------------------------------------------------
+# VLM prefill (Gemma-style stack over the prefix embeddings)
+# ---------------------------------------------------------------------------
+
+def prefill_weight_names(pcfg: PrefillShape, layers=None) -> List[Tuple[str, Tuple[int, ...]]]:
+    """(name, shape) of the prefill stack's parameters (the expert's layer
+    names), for all layers or the given ones."""
+    w, f = pcfg.width, pcfg.mlp_dim
+    out = []
+    for l in (range(pcfg.n_layers) if layers is None else layers):
+        p = f"layers.{l}."
+        out += [
+            (p + "attn_norm.g", (w,)),
+            (p + "q_proj.w", (pcfg.q_dim, w)),
+            (p + "k_proj.w", (pcfg.kv_dim, w)),
+            (p + "v_proj.w", (pcfg.kv_dim, w)),
+            (p + "o_proj.w", (w, pcfg.q_dim)),
+            (p + "mlp_norm.g", (w,)),
+            (p + "gate_proj.w", (f, w)),
+            (p + "up_proj.w", (f, w)),
+            (p + "down_proj.w", (w, f)),
+        ]
+    return out
+
+
+def make_prefill_weights(pcfg: PrefillShape, layers=None, seed: int | None = None) -> Dict[str, np.ndarray]:
+    """Prefill-stack parameters ~ N(0, 0.02) as float32 arrays (bf16 values in
+    a bf16 stack), for all layers or the given ones (each tensor has its own
+    stream, so a subset equals the same entries of the whole)."""
+    seed = pcfg.seed if seed is None else seed
+    ws: Dict[str, np.ndarray] = {}
+    for name, shape in prefill_weight_names(pcfg, layers):
+        a = _normal(seed, "vlm." + name, shape, pcfg.weight_std)
+        if pcfg.dtype == "bf16" and len(shape) == 2:
+            a = round_to_bf16(a)
+        ws[name] = a
+    return ws
+
+
+def make_prefix_embeddings(pcfg: PrefillShape, n_tokens: int | None = None, seed: int | None = None) -> np.ndarray:
+    """Prefix embeddings [P][w] ~ N(0,1) (bf16 values in a bf16 stack): the
+    stand-in for the vision tokens and text embeddings of one observation."""
+    seed = pcfg.seed if seed is None else seed
+    p = pcfg.n_tokens if n_tokens is None else n_tokens
+    x = _normal(seed, "prefix_embeddings", (p, pcfg.width), 1.0)
+    if pcfg.dtype == "bf16":
         x = round_to_bf16(x)
     return x

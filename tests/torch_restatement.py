@@ -117,3 +117,29 @@ def draft(W, dcfg, vis):
     gate = F.gelu(F.linear(u, _t(W["gate_proj.w"])), approximate="tanh")
     h = h + F.linear(gate * F.linear(u, _t(W["up_proj.w"])), _t(W["down_proj.w"]))
     return F.linear(h[:, v_len:], _t(W["action_head.w"]), _t(W["action_head.b"])).numpy()
+
+
+def prefill_kv(W, pcfg, emb):
+    """KV cache [L][2][1][P][Hkv][D] of the prefill stack over emb [P][w];
+    the whole prefix attends to itself without a mask."""
+    h = _t(emb)[None]                       # [1, P, w]
+    p_len, w = h.shape[1], h.shape[2]
+    hq, hkv, d = pcfg.n_q_heads, pcfg.n_kv_heads, pcfg.head_dim
+    pos = torch.arange(p_len)
+    out = torch.zeros(pcfg.n_layers, 2, 1, p_len, hkv, d, dtype=T64)
+    for l in range(pcfg.n_layers):
+        p = f"layers.{l}."
+        u = F.rms_norm(h, (w,), weight=1.0 + _t(W[p + "attn_norm.g"]), eps=pcfg.rms_eps)
+        k = rope_complex(F.linear(u, _t(W[p + "k_proj.w"])).view(1, p_len, hkv, d), pos, pcfg.rope_theta)
+        v = F.linear(u, _t(W[p + "v_proj.w"])).view(1, p_len, hkv, d)
+        out[l, 0] = k
+        out[l, 1] = v
+        q = rope_complex(F.linear(u, _t(W[p + "q_proj.w"])).view(1, p_len, hq, d), pos, pcfg.rope_theta)
+        rep = hq // hkv
+        o = F.scaled_dot_product_attention(q.transpose(1, 2), k.transpose(1, 2).repeat_interleave(rep, dim=1),
+                                           v.transpose(1, 2).repeat_interleave(rep, dim=1))
+        h = h + F.linear(o.transpose(1, 2).reshape(1, p_len, hq * d), _t(W[p + "o_proj.w"]))
+        u = F.rms_norm(h, (w,), weight=1.0 + _t(W[p + "mlp_norm.g"]), eps=pcfg.rms_eps)
+        gate = F.gelu(F.linear(u, _t(W[p + "gate_proj.w"])), approximate="tanh")
+        h = h + F.linear(gate * F.linear(u, _t(W[p + "up_proj.w"])), _t(W[p + "down_proj.w"]))
+    return out.numpy()
