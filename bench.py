@@ -6,6 +6,7 @@ bandwidth it achieves.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     python bench.py --workload flash-draft      # the FLASH draft model alone
+    python bench.py --workload gemma2b-prefill  # VLM prefill + the pi0-bf16 chunk, one graph
 
 One "step" is one call of rtv_denoise: the whole hot path (10 Euler steps
 through the expert) over one batch of synthetic input.  With N > 1 the
@@ -38,6 +39,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "10-step action-chunk latency (us) and achieved HBM GB/s vs 8 TB/s roofline"
+PREFILL_METRIC = ("prefill + 10-step chunk latency (us): Gemma-2B-class prefill over 816 tokens writing the "
+                  "KV cache, then the pi0-bf16 chunk, one CUDA graph")
 DRAFT_METRIC = "FLASH draft forward latency (us): one Gemma-2B-width block + action head over 768 image tokens"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
@@ -598,6 +601,137 @@ def run_draft(args, info):
     print(json.dumps(line), flush=True)
 
 
+def prefill_weights_bits(pc):
+    """The stack's parameters with matrices as bf16 bits, one layer at a time."""
+    from synthetic import f32_to_bf16_bits, make_prefill_weights
+    out = {}
+    for l in range(pc.n_layers):
+        for k, v in make_prefill_weights(pc, layers=[l]).items():
+            out[k] = f32_to_bf16_bits(v) if v.ndim == 2 else v
+    return out
+
+
+def run_prefill(args, info):
+    """Gemma-2B-class prefill over 816 embedding tokens writing the pi0-bf16
+    expert's KV cache, then its 10-step chunk, as one CUDA graph (one step =
+    one rtv_prefill_denoise).  Also times the prefill alone (rtv_prefill_kv)
+    for its tensor-pipe roofline."""
+    import torch
+
+    from flow_matching_action_dm0_b200 import ActionExpert, PrefillStack
+    from flow_matching_action_dm0_b200 import replicas as R
+    from synthetic import (f32_to_bf16_bits, get_config, get_prefill_config, make_noise, make_prefix_embeddings,
+                           make_state, make_weights)
+
+    dev = info.local_rank
+    torch.cuda.set_device(dev)
+    pc = get_prefill_config(args.workload)
+    cfg = get_config("pi0-bf16", n_steps=args.n_steps, prefix_len=pc.n_tokens)
+    if args.layers > 0:
+        pc = pc.with_(n_layers=args.layers)
+        cfg = cfg.with_(n_layers=args.layers)
+    n = cfg.n_steps
+    ex = ActionExpert(cfg, device=dev, max_batch=1, max_taus=4)
+    ex.load(make_weights(cfg))
+    pf = PrefillStack(pc, device=dev)
+    pf.load(prefill_weights_bits(pc))
+    emb = make_prefix_embeddings(pc)
+    emb_t = torch.from_numpy(f32_to_bf16_bits(emb).view(np.int16)).view(torch.bfloat16)
+    emb_d = emb_t.cuda(dev)
+    noise, state = make_noise(cfg)[0], make_state(cfg)[0]
+    noise_d, state_d = torch.from_numpy(noise).cuda(dev), torch.from_numpy(state).cuda(dev)
+    out_d = torch.empty_like(noise_d)
+    stream = torch.cuda.Stream(dev)
+    for _ in range(max(3, args.warmup)):
+        pf.denoise(ex, emb_d, noise_d, state_d, n, out_d, stream=stream)
+        pf.kv(ex, emb_d, stream=stream)
+    torch.cuda.synchronize(dev)
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    gpu_id = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    K = args.steps
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    R.barrier(info, dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(gpu_id) as clk:
+        start.record(stream)
+        for _ in range(K):
+            pf.denoise(ex, emb_d, noise_d, state_d, n, out_d, stream=stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    R.barrier(info, dev)
+    ms = R.max_over_ranks(start.elapsed_time(end) / K, info, dev)
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    for _ in range(K):
+        pf.kv(ex, emb_d, stream=stream)
+    p1.record(stream)
+    torch.cuda.synchronize(dev)
+    prefill_ms = R.max_over_ranks(p0.elapsed_time(p1) / K, info, dev)
+    for h in (pf, ex):
+        s, bits = h.status()
+        if s != 0:
+            raise RuntimeError(f"device status {bits:#x} after the timed region")
+    emb_h = emb_t.pin_memory()
+    noise_h = torch.from_numpy(noise).pin_memory()
+    state_h = torch.from_numpy(state).pin_memory()
+    out_h = torch.empty_like(noise_h).pin_memory()
+    pf.denoise(ex, emb_h, noise_h, state_h, n, out_h, stream=stream)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        pf.denoise(ex, emb_h, noise_h, state_h, n, out_h, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = R.max_over_ranks(e0.elapsed_time(e1) / K, info, dev)
+    kernels = pf.kernels_per_call(pc.n_tokens, n)
+    pf.close()
+    ex.close()
+    if not info.is_main:
+        return
+    peaks, peak_kind = load_peaks()
+    flops = pc.flops()
+    achieved = flops / (prefill_ms * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    line = {
+        "metric": PREFILL_METRIC, "value": ms * 1000.0, "unit": "us", "n_gpus": info.world, "steps": K,
+        "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload if args.layers <= 0 else f"{args.workload} ({pc.n_layers} layers)",
+                   "n_tokens": pc.n_tokens, "prefill_layers": pc.n_layers, "prefill_width": pc.width,
+                   "prefill_mlp": pc.mlp_dim, "expert": "pi0-bf16", "n_steps": n, "batch": 1,
+                   "parallelism": f"replicas x{info.world}",
+                   "l2": "inputs larger than L2: 3.7 GB of stack weights and 623 MB of expert weights per call; "
+                         "no flush"},
+        "prefill_us": prefill_ms * 1000.0,
+        "roofline": {"bound": "tensor", "kernel": "whole prefill graph (rtv_prefill_kv)", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_kind": f"{peak_kind} bf16_tflops_sustained", "algorithmic_flops_per_launch": flops,
+                     "traffic": None},
+        "e2e": {"value": e2e_ms * 1000.0, "unit": "us",
+                "h2d_bytes_per_step": int(emb_t.numel() * 2 + noise.nbytes + state.nbytes),
+                "d2h_bytes_per_step": int(noise.nbytes)},
+        "clocks": clk.summary(),
+        "gpu_launches": int(kernels * K) if kernels > 0 else None,
+    }
+    if info.world == 1 and not args.no_cpu_baseline:
+        from oracle import expert as O
+        from oracle import prefill as OP
+        from synthetic import make_prefill_weights
+        one = pc.with_(n_layers=2)
+        t0 = time.perf_counter()
+        OP.prefill_kv(lambda l: make_prefill_weights(one, layers=[l]), one, emb)
+        t_two = time.perf_counter() - t0
+        per_step_s, k = oracle_step_seconds(cfg, args.cpu_seconds / 2)
+        line["cpu_baseline"] = {
+            "value": (t_two * (pc.n_layers - 1) + per_step_s * n) * 1e6, "unit": "us", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"a 2-layer oracle prefill over {pc.n_tokens} tokens (one full layer + one K/V layer, "
+                      f"weight generation included) scaled to {pc.n_layers} layers, plus {k} oracle Euler steps "
+                      f"scaled x{n}"}
+    print(json.dumps(line), flush=True)
+
+
 def run_trace(args):
     """One traced chunk: the library prints per-CTA phase stamps (globaltimer)
     of the projections and the attention of layer 0, first Euler step."""
@@ -627,10 +761,12 @@ def main(argv=None):
         run_reference(args, info)
         return 0
     info = R.init("nccl" if info.world > 1 else "gloo")
-    from synthetic import DRAFTS
+    from synthetic import DRAFTS, PREFILLS
     try:
         if args.workload in DRAFTS:
             run_draft(args, info)
+        elif args.workload in PREFILLS:
+            run_prefill(args, info)
         else:
             run_ours(args, info)
     finally:

@@ -28,7 +28,8 @@ EXPORTS = ("rtv_create", "rtv_load_expert", "rtv_set_prefix_kv", "rtv_denoise", 
            "rtv_device_status", "rtv_last_error", "rtv_path_name", "rtv_graph_kernel_count", "rtv_destroy",
            "rtv_set_prefix_kv_static", "rtv_draft_create", "rtv_draft_load", "rtv_draft_forward", "rtv_flash_round",
            "rtv_draft_device_status", "rtv_draft_last_error", "rtv_draft_path_name", "rtv_draft_kernel_count",
-           "rtv_draft_destroy")
+           "rtv_draft_destroy", "rtv_prefill_create", "rtv_prefill_load", "rtv_prefill_kv", "rtv_prefill_denoise",
+           "rtv_prefill_device_status", "rtv_prefill_last_error", "rtv_prefill_kernel_count", "rtv_prefill_destroy")
 
 
 class rtv_expert_config(C.Structure):
@@ -47,6 +48,14 @@ class rtv_draft_config(C.Structure):
         ("mlp_dim", C.c_int), ("n_queries", C.c_int), ("action_dim", C.c_int), ("max_vis", C.c_int),
         ("max_batch", C.c_int), ("dtype", C.c_int), ("rms_eps", C.c_float), ("rope_theta", C.c_float),
         ("barrier_timeout_ns", C.c_longlong),
+    ]
+
+
+class rtv_prefill_config(C.Structure):
+    _fields_ = [
+        ("n_layers", C.c_int), ("width", C.c_int), ("n_q_heads", C.c_int), ("n_kv_heads", C.c_int),
+        ("head_dim", C.c_int), ("mlp_dim", C.c_int), ("max_tokens", C.c_int), ("dtype", C.c_int),
+        ("rms_eps", C.c_float), ("rope_theta", C.c_float), ("barrier_timeout_ns", C.c_longlong),
     ]
 
 
@@ -103,9 +112,21 @@ def load_library(path: str = LIB_PATH):
     lib.rtv_draft_kernel_count.restype = I
     lib.rtv_draft_destroy.argtypes = [P]
     lib.rtv_draft_destroy.restype = None
+    lib.rtv_prefill_create.argtypes = [C.POINTER(rtv_prefill_config), I, C.POINTER(P)]
+    lib.rtv_prefill_load.argtypes = [P, C.POINTER(rtv_tensor), I]
+    lib.rtv_prefill_kv.argtypes = [P, P, P, I, P]
+    lib.rtv_prefill_denoise.argtypes = [P, P, P, I, P, P, I, P, P]
+    lib.rtv_prefill_device_status.argtypes = [P, U]
+    lib.rtv_prefill_last_error.argtypes = [P]
+    lib.rtv_prefill_last_error.restype = C.c_char_p
+    lib.rtv_prefill_kernel_count.argtypes = [P, I, I]
+    lib.rtv_prefill_kernel_count.restype = I
+    lib.rtv_prefill_destroy.argtypes = [P]
+    lib.rtv_prefill_destroy.restype = None
     for n in ("rtv_create", "rtv_load_expert", "rtv_set_prefix_kv", "rtv_set_prefix_kv_static", "rtv_denoise",
               "rtv_verify", "rtv_device_status", "rtv_draft_create", "rtv_draft_load", "rtv_draft_forward",
-              "rtv_flash_round", "rtv_draft_device_status"):
+              "rtv_flash_round", "rtv_draft_device_status", "rtv_prefill_create", "rtv_prefill_load",
+              "rtv_prefill_kv", "rtv_prefill_denoise", "rtv_prefill_device_status"):
         getattr(lib, n).restype = I
     _lib = lib
     return lib
@@ -235,3 +256,55 @@ def rtv_draft_kernel_count(d, n_vis: int, batch: int) -> int:
 def rtv_draft_destroy(d):
     if d:
         load_library().rtv_draft_destroy(d)
+
+
+# VLM prefill -------------------------------------------------------------------
+
+def rtv_prefill_create(cfg: rtv_prefill_config, device: int = 0):
+    lib = load_library()
+    h = C.c_void_p()
+    s = lib.rtv_prefill_create(C.byref(cfg), int(device), C.byref(h))
+    if s != RTV_OK:
+        raise RtvError(s, "rtv_prefill_create failed")
+    return h
+
+
+def _pcheck(p, s):
+    if s != RTV_OK:
+        raise RtvError(s, load_library().rtv_prefill_last_error(p).decode())
+    return s
+
+
+def rtv_prefill_load(p, tensors):
+    arr = (rtv_tensor * len(tensors))(*tensors)
+    return _pcheck(p, load_library().rtv_prefill_load(p, arr, len(tensors)))
+
+
+def rtv_prefill_kv(p, h, emb_ptr: int, n_tokens: int, stream: int = 0):
+    return _pcheck(p, load_library().rtv_prefill_kv(p, h, C.c_void_p(emb_ptr), int(n_tokens), C.c_void_p(stream)))
+
+
+def rtv_prefill_denoise(p, h, emb_ptr: int, n_tokens: int, noise_ptr: int, state_ptr: int, n_steps: int,
+                        out_ptr: int, stream: int = 0):
+    return _pcheck(p, load_library().rtv_prefill_denoise(
+        p, h, C.c_void_p(emb_ptr), int(n_tokens), C.c_void_p(noise_ptr), C.c_void_p(state_ptr), int(n_steps),
+        C.c_void_p(out_ptr), C.c_void_p(stream)))
+
+
+def rtv_prefill_device_status(p):
+    bits = C.c_uint(0)
+    s = load_library().rtv_prefill_device_status(p, C.byref(bits))
+    return s, bits.value
+
+
+def rtv_prefill_last_error(p) -> str:
+    return load_library().rtv_prefill_last_error(p).decode()
+
+
+def rtv_prefill_kernel_count(p, n_tokens: int, n_steps: int = 0) -> int:
+    return int(load_library().rtv_prefill_kernel_count(p, int(n_tokens), int(n_steps)))
+
+
+def rtv_prefill_destroy(p):
+    if p:
+        load_library().rtv_prefill_destroy(p)

@@ -37,6 +37,13 @@ rtv_status fast_block_prefix(rtv_ctx* ctx, const __nv_bfloat16* vis, int n_vis, 
 // Bare block: residual stream of G suffixes set to rows[t % n_src_rows]
 // (fp32, [n_src_rows][width]) with the first norm's inputs.
 rtv_status fast_block_embed(rtv_ctx* ctx, const float* rows, int n_src_rows, int G, cudaStream_t st);
+// Prefill (pre: a bare block stack whose suffix is a group of 64 query rows):
+// the stack over P tokens given as bf16 embeddings emb [P][width], writing
+// every layer's keys (RoPE at positions 0..P-1) and values into the prefix
+// cache of the expert ex (batch element 0) and its tensor-core tiles; the
+// last layer computes keys and values only.  rope_cs / rope_sn: [P][D/2].
+rtv_status fast_prefill(rtv_ctx* pre, rtv_ctx* ex, const __nv_bfloat16* emb, int P, const float* rope_cs,
+                        const float* rope_sn, cudaStream_t st);
 void fast_destroy(rtv_ctx* ctx);
 // Diagnostic phase trace (only when the RTV_TRACE environment variable is set).
 void fast_arm_trace(rtv_ctx* ctx);

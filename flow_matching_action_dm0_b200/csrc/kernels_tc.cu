@@ -55,6 +55,10 @@ namespace rtv {
 
 enum { GM_QKV = 0, GM_O = 1, GM_GU = 2, GM_DOWN = 3 };
 
+// Attention mask of query rows that form a prefix attending to itself: the
+// keys are the cached prefix only (internal; after the RTV_MASK_* values).
+constexpr int kMaskPrefixOnly = 2;
+
 // Element offset of (row t, column k) of a bf16 operand [rows][K] stored
 // tiled and pre-swizzled: blocks of `block_rows` rows x 64 columns (128-byte
 // rows, stacked densely), and inside a block the eight 16-byte chunks of row
@@ -111,7 +115,10 @@ struct GemmArgs {
   int T, n_mma, kslice, stages, w, S, Hq, Hkv, D, F, K, w_tile0;
   int tt;                     // token rows per CTA (a multiple of 16, <= 256); blockIdx.z picks the tile
   int nt_base;                // first 128-row weight tile of the grid within the layer (QKV: K/V tiles only)
-  int kv_rows;                // row stride of ks / vs per (suffix, kv head) when qt is not set
+  int kv_rows;                // row stride of ks / vs per (sequence, kv head)
+  int seq;                    // QKV: tokens of one sequence -- RoPE position and ks/vs row are t % seq, the
+                              // sequence t / seq (= S for suffixes; the prefix length for a prefix)
+  int kv_prefix;              // QKV with qt set: keys and values still go to ks / vs rows, not to kts / vts
   float eps;
 };
 
@@ -372,7 +379,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
     } else if (rope) {
       for (int c = tid; c < n_own * 32; c += kEpiThreads) {
         const int tl = c >> 5, ch = c & 31;   // chunks 0-15: cos, 16-31: sin (64 floats each)
-        const int s = (t0 + t_own0 + tl) % a.S;
+        const int s = (t0 + t_own0 + tl) % a.seq;   // position in its sequence
         const float* src = (ch < 16 ? a.rope_cs : a.rope_sn) + (size_t)s * hd + dq0 + (ch & 15) * 4;
         ptx::cp_async_16(in_a + (uint32_t)(c * 16), src);
       }
@@ -510,7 +517,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
           *reinterpret_cast<uint32_t*>(a.m + ts_offset(t, nt * 64 + f0, n_rows)) =
               ptx::pack_bf16x2(gelu_tanh(x1.x) * x2.x, gelu_tanh(x1.y) * x2.y);
         } else {
-          const int g = t / a.S, s = t - g * a.S;
+          const int g = t / a.S, s = t - g * a.S;           // suffix group and row (q and suffix K/V tiles)
+          const int sq = t / a.seq, sp = t - sq * a.seq;    // sequence and position (K/V rows)
           float2 y1 = x1, y2 = x2;
           if (rope) {
             const float2 c = *reinterpret_cast<const float2*>(in_s + tl * 128 + f0);
@@ -519,7 +527,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
             y2 = make_float2(x2.x * c.x + x1.x * sn.x, x2.y * c.y + x1.y * sn.y);
           }
           const int d1 = dq0 + f0, d2 = d1 + hd;
-          if (a.qt) {
+          if (a.qt && (hh < a.Hq || !a.kv_prefix)) {
             if (hh < a.Hq) {
               __nv_bfloat16* dst = a.qt + (size_t)(g * (a.Hq >> 1) + (hh >> 1)) * 128 * a.D;
               const int row = ((hh & 1) << 6) + s;
@@ -539,8 +547,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
           } else {
             __nv_bfloat16* dst;
             if (hh < a.Hq) dst = a.q + ((size_t)t * a.Hq + hh) * a.D;
-            else if (hh < a.Hq + a.Hkv) dst = a.ks + (((size_t)g * a.Hkv + (hh - a.Hq)) * a.kv_rows + s) * a.D;
-            else dst = a.vs + (((size_t)g * a.Hkv + (hh - a.Hq - a.Hkv)) * a.kv_rows + s) * a.D;
+            else if (hh < a.Hq + a.Hkv) dst = a.ks + (((size_t)sq * a.Hkv + (hh - a.Hq)) * a.kv_rows + sp) * a.D;
+            else dst = a.vs + (((size_t)sq * a.Hkv + (hh - a.Hq - a.Hkv)) * a.kv_rows + sp) * a.D;
             *reinterpret_cast<uint32_t*>(dst + d1) = ptx::pack_bf16x2(y1.x, y1.y);
             *reinterpret_cast<uint32_t*>(dst + d2) = ptx::pack_bf16x2(y2.x, y2.y);
           }
@@ -975,7 +983,8 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const AttnTcArgs a) {
   const int r = 32 * quarter + lane;
   const int s = r & 63;
   const bool row_valid = s < a.S;
-  const int n_keys = suffix_tile ? a.S : min(64, a.P - 64 * rank);
+  // (a prefix attending to itself has no suffix keys: its suffix rank adds nothing)
+  const int n_keys = suffix_tile ? (a.mask_mode == kMaskPrefixOnly ? 0 : a.S) : min(64, a.P - 64 * rank);
   // the Pi0 block mask hides the action tokens of the suffix from the state token (row s == 0)
   const int n_vis = (a.mask_mode == RTV_MASK_PI0_BLOCK && suffix_tile && s == 0) ? 1 : n_keys;
   if (!ptx::mbar_wait(&bars[2], 0, a.timeout_ns)) atomicOr(a.status, RTV_DEV_TIMEOUT);
@@ -1971,6 +1980,7 @@ rtv_status fast_block_prefix(rtv_ctx* ctx, const __nv_bfloat16* vis, int n_vis, 
   a.ks = (__nv_bfloat16*)ctx->prefix_kv;
   a.vs = a.ks + kv_layer;
   a.kv_rows = k.max_prefix_len;
+  a.seq = n_vis;
   a.rope_cs = rope_cs;
   a.rope_sn = rope_sn;
   a.status = ctx->status;
@@ -2004,6 +2014,159 @@ rtv_status fast_block_embed(rtv_ctx* ctx, const float* rows, int n_src_rows, int
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     ctx->last_error = std::string("block input launch: ") + cudaGetErrorString(e);
+    return RTV_ERR_CUDA;
+  }
+  return RTV_OK;
+}
+
+rtv_status fast_prefill(rtv_ctx* pre, rtv_ctx* ex, const __nv_bfloat16* emb, int P, const float* rope_cs,
+                        const float* rope_sn, cudaStream_t st) {
+  FastPath* fp = pre->fast;
+  FastPath* xp = ex->fast;
+  const rtv_expert_config& k = pre->cfg;
+  const rtv_expert_config& kx = ex->cfg;
+  const int w = k.width, F = k.mlp_dim, D = k.head_dim, Q = pre->Q, KV = pre->KV, L = k.n_layers;
+  const int S = pre->S;                       // query rows per attention group (64)
+  const int G = (P + S - 1) / S;              // query groups
+  const int T = P, n_mma = G * S;             // real token rows; rows of the tiled layouts
+  if (!fp || !xp || !xp->tc_attn || !fp->tc_attn || G > pre->Gmax || S != 64 || (P + 63) / 64 + 1 > 16 ||
+      (P + 63) / 64 > xp->ntile_max) {
+    pre->last_error = "prefill shape not supported by the tensor-core path";
+    return RTV_ERR_UNSUPPORTED;
+  }
+  int n_tt = 1, tt = 16;
+  token_tiles(n_mma, &n_tt, &tt);
+  const int T_tile = std::min(T, tt);
+  const int nq = Q + 2 * KV;
+  const GemmPlan p_qkv = plan_gemm(fp, nq, w, tt, T_tile, true, false, n_tt);
+  const GemmPlan p_kv = plan_gemm(fp, 2 * KV, w, tt, T_tile, true, false, n_tt);
+  const GemmPlan p_o = plan_gemm(fp, w, Q, tt, T_tile, true, false, n_tt);
+  const GemmPlan p_gu = plan_gemm(fp, 2 * F, w, tt, T_tile, false, false, n_tt);
+  const GemmPlan p_dn = plan_gemm(fp, w, F, tt, T_tile, true, false, n_tt);
+  if (!(p_qkv.valid && p_kv.valid && p_o.valid && p_gu.valid && p_dn.valid)) {
+    pre->last_error = "no tensor-core split fits the prefill";
+    return RTV_ERR_UNSUPPORTED;
+  }
+  if (getenv("RTV_LOG")) {
+    const GemmPlan* pls[5] = {&p_qkv, &p_kv, &p_o, &p_gu, &p_dn};
+    const char* nm[5] = {"qkv", "kv", "o", "gu", "down"};
+    for (int i = 0; i < 5; ++i)
+      fprintf(stderr, "[rtv] prefill T=%d %s: tiles=%d token_tiles=%d cluster=%d kslice=%d stages=%d smem=%d\n", T,
+              nm[i], pls[i]->n_tiles, pls[i]->n_tt, pls[i]->cs, pls[i]->kslice, pls[i]->stages, pls[i]->smem);
+  }
+  // layer 0's norm input and residual from the embeddings
+  norm_input_kernel<__nv_bfloat16><<<T, 128, 0, st>>>(emb, T, pre->h, pre->W.layers[0].g_attn, fp->hb, fp->ssp,
+                                                       n_mma, w);
+  cudaError_t e = cudaGetLastError();
+
+  GemmArgs base{};
+  base.h = pre->h;
+  base.hb = fp->hb;
+  base.ssp = fp->ssp;
+  base.qt = fp->qt;
+  base.kts = fp->kts;
+  base.vts = fp->vts;
+  base.rope_cs = rope_cs;
+  base.rope_sn = rope_sn;
+  base.m = fp->mb;
+  base.status = pre->status;
+  base.timeout_ns = k.barrier_timeout_ns;
+  base.T = T;
+  base.n_mma = n_mma;
+  base.tt = tt;
+  base.kv_rows = kx.max_prefix_len;
+  base.seq = P;
+  base.kv_prefix = 1;
+  base.w = w;
+  base.S = S;
+  base.Hq = k.n_q_heads;
+  base.Hkv = k.n_kv_heads;
+  base.D = D;
+  base.F = F;
+  base.eps = k.rms_eps;
+
+  AttnTcArgs atc{};
+  atc.qt = fp->qt;
+  atc.kts = fp->kts;
+  atc.vts = fp->vts;
+  atc.o = fp->ob;
+  atc.part_o = fp->att_po;
+  atc.part_ml = fp->att_pml;
+  atc.status = pre->status;
+  atc.timeout_ns = k.barrier_timeout_ns;
+  atc.S = S;
+  atc.P = P;
+  atc.Hq = k.n_q_heads;
+  atc.Hkv = k.n_kv_heads;
+  atc.pbs = 0;                      // every query group reads the one prefix
+  atc.mask_mode = kMaskPrefixOnly;
+  atc.ntile_max = xp->ntile_max;
+  atc.n_mma = n_mma;
+  atc.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+  const int ntp = (P + 63) / 64;
+  const size_t kv_layer = (size_t)kx.max_batch * kx.n_kv_heads * kx.max_prefix_len * D;
+  const size_t ptile_layer = (size_t)kx.max_batch * kx.n_kv_heads * xp->ntile_max * 64 * D;
+
+  for (int l = 0; l < L && e == cudaSuccess; ++l) {
+    const bool last = l == L - 1;
+    __nv_bfloat16* kl = (__nv_bfloat16*)ex->prefix_kv + (size_t)(2 * l) * kv_layer;
+    // q/k/v of the layer (the last layer: keys and values only, straight
+    // into the expert's cache), RoPE at positions 0..P-1
+    GemmArgs a = base;
+    a.wt = fp->w_qkv;
+    a.act = fp->hb;
+    a.K = w;
+    a.w_tile0 = l * nq / 128;
+    a.nt_base = last ? Q / 128 : 0;
+    a.ks = kl;
+    a.vs = kl + kv_layer;
+    a.pf = last ? nullptr : (const uint8_t*)(fp->w_o + (size_t)l * w * Q);
+    a.pf_bytes = last ? 0 : (unsigned long long)w * Q * 2;
+    e = launch_gemm<GM_QKV>(a, last ? p_kv : p_qkv, st, fp->pf_cap);
+    // the layer's cache in the attention's tiles (the expert reads them too)
+    if (e == cudaSuccess) {
+      prefix_tile_kernel<<<4 * fp->num_sms, 256, 0, st>>>(kl, xp->pkt + (size_t)l * ptile_layer,
+                                                         xp->pvt + (size_t)l * ptile_layer, 1, 1, P, k.n_kv_heads,
+                                                         D, kx.max_batch, kx.max_prefix_len, xp->ntile_max);
+      e = cudaGetLastError();
+    }
+    if (last) break;
+    atc.pkt = xp->pkt + (size_t)l * ptile_layer;
+    atc.pvt = xp->pvt + (size_t)l * ptile_layer;
+    if (e == cudaSuccess)
+      e = D == 256 ? launch_attn_tc<256>(atc, ntp + 1, G, st) : launch_attn_tc<128>(atc, ntp + 1, G, st);
+
+    a = base;
+    a.wt = fp->w_o;
+    a.act = fp->ob;
+    a.K = Q;
+    a.w_tile0 = l * w / 128;
+    a.pf = (const uint8_t*)(fp->w_gu + (size_t)l * 2 * F * w);
+    a.pf_bytes = (unsigned long long)2 * F * w * 2;
+    a.g_next = pre->W.layers[l].g_mlp;
+    if (e == cudaSuccess) e = launch_gemm<GM_O>(a, p_o, st, fp->pf_cap);
+
+    a = base;
+    a.wt = fp->w_gu;
+    a.act = fp->hb;
+    a.K = w;
+    a.w_tile0 = l * 2 * F / 128;
+    a.pf = (const uint8_t*)(fp->w_down + (size_t)l * w * F);
+    a.pf_bytes = (unsigned long long)w * F * 2;
+    if (e == cudaSuccess) e = launch_gemm<GM_GU>(a, p_gu, st, fp->pf_cap);
+
+    a = base;
+    a.wt = fp->w_down;
+    a.act = fp->mb;
+    a.K = F;
+    a.w_tile0 = l * w / 128;
+    a.pf = (const uint8_t*)(fp->w_qkv + (size_t)(l + 1) * nq * w);
+    a.pf_bytes = (unsigned long long)nq * w * 2;
+    a.g_next = pre->W.layers[l + 1].g_attn;
+    if (e == cudaSuccess) e = launch_gemm<GM_DOWN>(a, p_dn, st, fp->pf_cap);
+  }
+  if (e != cudaSuccess) {
+    pre->last_error = std::string("prefill launch: ") + cudaGetErrorString(e);
     return RTV_ERR_CUDA;
   }
   return RTV_OK;
@@ -2060,6 +2223,7 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
   base.n_mma = n_mma;
   base.tt = tt;
   base.kv_rows = S;
+  base.seq = S;
   base.w = w;
   base.S = S;
   base.Hq = k.n_q_heads;

@@ -142,7 +142,8 @@ enum { KIND_DENOISE = 0, KIND_VERIFY = 1 };
 // Precompute the input-independent tables of a graph (time condition of the
 // Euler schedule, RoPE table of the suffix positions), then capture.
 template <typename WT>
-rtv_status build_graph(rtv_ctx* ctx, int kind, int n, int batch, int P, GraphEntry& ge) {
+rtv_status build_graph(rtv_ctx* ctx, int kind, int n, int batch, int P, GraphEntry& ge,
+                       const GraphPrologue* prologue = nullptr) {
   const rtv_expert_config& k = ctx->cfg;
   cudaStream_t st = ctx->cap_stream;
   const int S = ctx->S, D = k.head_dim, w = k.width;
@@ -169,6 +170,7 @@ rtv_status build_graph(rtv_ctx* ctx, int kind, int n, int batch, int P, GraphEnt
   auto chain = [&](rtv_status s2) {
     if (fs == RTV_OK) fs = s2;
   };
+  if (prologue) chain((*prologue)(st));
   if (kind == KIND_DENOISE) {
     const float dt = (float)(1.0 / (double)n);
     if (ctx->use_fast) {
@@ -247,6 +249,21 @@ rtv_status get_graph(rtv_ctx* ctx, int kind, int n, int batch, GraphEntry** out)
 }  // namespace
 
 namespace rtv {
+
+rtv_status capture_denoise(rtv_ctx* ctx, int n_steps, int P, const GraphPrologue& prologue, GraphEntry& ge) {
+  if (!ctx->use_fast || ctx->cfg.dtype != RTV_BF16)
+    return fail(ctx, RTV_ERR_UNSUPPORTED, "capture with a prologue needs the tensor-core path");
+  const rtv_status s = build_graph<__nv_bfloat16>(ctx, KIND_DENOISE, n_steps, 1, P, ge, &prologue);
+  if (s != RTV_OK) {
+    for (void* p : ge.owned) cudaFree(p);
+    ge.owned.clear();
+    if (ge.exec) cudaGraphExecDestroy(ge.exec);
+    if (ge.graph) cudaGraphDestroy(ge.graph);
+    ge.exec = nullptr;
+    ge.graph = nullptr;
+  }
+  return s;
+}
 
 rtv_status ctx_create(const rtv_expert_config& k, int cuda_device, int S, bool block_only, rtv_ctx** out) {
   *out = nullptr;

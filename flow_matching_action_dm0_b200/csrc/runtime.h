@@ -4,6 +4,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <functional>
 #include <map>
 #include <string>
 #include <tuple>
@@ -58,6 +59,9 @@ struct ParamSlot {
 };
 using SlotTable = std::unordered_map<std::string, ParamSlot>;
 
+// Work captured at the head of a graph, before the denoising loop.
+using GraphPrologue = std::function<rtv_status(cudaStream_t)>;
+
 }  // namespace rtv
 
 struct rtv_ctx {
@@ -105,6 +109,10 @@ void add_layer_slots(rtv_ctx* ctx, SlotTable& slots, const std::string& p, Layer
 // Validate a parameter list against the table (every name exactly once,
 // dtype and shape), then allocate and copy.  Nothing is allocated on a bad list.
 rtv_status load_slots(rtv_ctx* ctx, SlotTable& slots, const rtv_tensor* params, int n_params);
+// Capture (not launch) the denoising graph of n_steps Euler steps over a
+// prefix of P tokens (batch 1, tensor-core path) with `prologue` enqueued
+// first, on the context's capture stream, into ge.
+rtv_status capture_denoise(rtv_ctx* ctx, int n_steps, int P, const GraphPrologue& prologue, GraphEntry& ge);
 // The SIMT layers over G suffixes of ctx->S rows (residual stream ctx->h).
 template <typename WT>
 void simt_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, const float* rope_cs, const float* rope_sn,

@@ -293,6 +293,69 @@ int rtv_draft_kernel_count(rtv_draft* d, int n_vis, int batch);
 /* Release every resource of the draft model.  NULL is accepted. */
 void rtv_draft_destroy(rtv_draft* d);
 
+/* ------------------------------------------------------------------------
+ * VLM prefill ([DM0.5] 5.1: the prefix is encoded once into a per-layer KV
+ * cache; 6.5: one graph replay per request).
+ *
+ * A Gemma-style stack over the prefix embeddings of one observation (n_tokens
+ * rows of `width`): RMSNorm with gain 1+g, q/k/v projections, RoPE at
+ * positions 0..n_tokens-1, softmax attention in which every prefix token
+ * sees every prefix token, o_proj + residual, RMSNorm, GeGLU MLP + residual.
+ * Layer l's keys (after RoPE) and values become the expert's cached prefix
+ * of layer l, so the stack has the expert's n_layers, n_kv_heads and
+ * head_dim.  The last layer's attention output and MLP are not computed.
+ * bf16 only (tensor-core path).
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  int n_layers, width, n_q_heads, n_kv_heads, head_dim, mlp_dim;
+  int max_tokens;     /* largest n_tokens a call may pass (<= 960)                */
+  int dtype;          /* RTV_BF16                                                 */
+  float rms_eps;
+  float rope_theta;   /* 0 disables rotary embedding                              */
+  long long barrier_timeout_ns;   /* 0 = library default (100 ms)                 */
+} rtv_prefill_config;
+
+typedef struct rtv_prefill rtv_prefill;
+
+/* Create a prefill stack on CUDA device `cuda_device`.  width must be a
+ * multiple of 128.  Returns RTV_ERR_UNSUPPORTED for RTV_F32 or a shape the
+ * tensor-core path does not take.  *out is NULL on failure. */
+rtv_status rtv_prefill_create(const rtv_prefill_config* cfg, int cuda_device, rtv_prefill** out);
+
+/* Copy and pack the stack's parameters: for every layer l the names of
+ * rtv_load_expert's layers (layers.l.attn_norm.g, layers.l.q_proj.w, ...,
+ * layers.l.down_proj.w), matrices in bf16, gains in RTV_F32.  Synchronous. */
+rtv_status rtv_prefill_load(rtv_prefill* p, const rtv_tensor* params, int n_params);
+
+/* Run the stack over emb [n_tokens][width] (bf16, device or host) and
+ * install the result as the prefix KV cache of the expert `ctx` (batch 1,
+ * prefix_len = n_tokens), as rtv_set_prefix_kv would.  The expert must be a
+ * bf16 tensor-core context with the stack's n_layers, n_kv_heads and
+ * head_dim, and n_tokens <= its max_prefix_len.  Asynchronous on `stream`;
+ * the first call for a given n_tokens captures a CUDA graph. */
+rtv_status rtv_prefill_kv(rtv_prefill* p, rtv_ctx* ctx, const void* emb, int n_tokens, rtv_stream stream);
+
+/* Prefill followed by rtv_denoise(ctx, noise, state, n_steps) for one
+ * observation (batch 1), captured as ONE CUDA graph per (n_tokens, n_steps)
+ * and replayed: emb [n_tokens][width] bf16, noise [H][A], state [Sd],
+ * actions_out [H][A]; each device or host memory.  Leaves the prefix
+ * installed in ctx.  Asynchronous on `stream`. */
+rtv_status rtv_prefill_denoise(rtv_prefill* p, rtv_ctx* ctx, const void* emb, int n_tokens, const float* noise,
+                               const float* state, int n_steps, float* actions_out, rtv_stream stream);
+
+/* As rtv_device_status, for the stack's kernels. */
+rtv_status rtv_prefill_device_status(rtv_prefill* p, unsigned* bits);
+
+/* Last error message of the prefill stack (never NULL). */
+const char* rtv_prefill_last_error(rtv_prefill* p);
+
+/* Kernel launches of the graph captured for (n_tokens, n_steps); n_steps 0
+ * is rtv_prefill_kv's graph.  -1 before it has been captured. */
+int rtv_prefill_kernel_count(rtv_prefill* p, int n_tokens, int n_steps);
+
+/* Release every resource of the prefill stack.  NULL is accepted. */
+void rtv_prefill_destroy(rtv_prefill* p);
+
 #ifdef __cplusplus
 }
 #endif
