@@ -150,8 +150,14 @@ __host__ __device__ inline GemmSmem gemm_smem_layout(int stages, int n_mma, int 
   const int core = s.ring_bytes + (f8 ? stages * 8192 : 0);
   const int part_bytes = n_mma * 512;
   s.part_off = 0;   // the partial tile overlays the ring: every MMA has completed when it is written
-  s.recv_off = core > part_bytes ? core : part_bytes;
-  s.in_off = s.recv_off + cs * per * 512;   // [per][128] fp32 epilogue inputs of the owned tokens
+  if (cs == 1) {
+    // a lone CTA owns every token: its partial tile is its receive buffer
+    s.recv_off = s.part_off;
+    s.in_off = core > part_bytes ? core : part_bytes;
+  } else {
+    s.recv_off = core > part_bytes ? core : part_bytes;
+    s.in_off = s.recv_off + cs * per * 512;   // [per][128] fp32 epilogue inputs of the owned tokens
+  }
   s.bar_off = s.in_off + (with_in ? per * 512 : 0);   // GU reads no per-token epilogue inputs
   s.total = s.bar_off + (3 * stages + 2) * 8 + 16 + 1024;   // barriers, TMEM slot, alignment slack
   return s;
@@ -360,7 +366,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
     // ---- epilogue warps 2..9 ----
     const int tid = threadIdx.x - 64;
     ptx::pdl_wait();   // this role reads and writes what earlier kernels produced
-    if (tid == 0) ptx::mbar_expect_tx(rbar, (uint32_t)(cs * n_own * 512));
+    if (tid == 0 && cs > 1) ptx::mbar_expect_tx(rbar, (uint32_t)(cs * n_own * 512));
     // Everything the epilogue reads from global memory depends only on earlier
     // kernels, so it is requested now, while the MMAs run: the owned tokens'
     // residual rows of this tile (O, DOWN) or their RoPE cos/sin (QKV) go to
@@ -446,7 +452,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
     if (trace && tid == 0) trace[TR_PART] = ptx::globaltimer();
     cluster_wait();   // entry phase: every rank has started and initialised its barriers
     if (trace && tid == 0) trace[TR_ENTRY] = ptx::globaltimer();
-    if (tid < cs) {   // one lane per destination rank
+    if (cs > 1 && tid < cs) {   // one lane per destination rank
       const int r = tid;
       const uint32_t part_a = ptx::smem_u32(part), recv_a = ptx::smem_u32(recv), rbar_a = ptx::smem_u32(rbar);
       const int o0 = r * per, no = max(0, min(T, o0 + per) - o0);
@@ -458,7 +464,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
     ptx::cp_async_wait_all();
     asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
     if (trace && tid == 0) trace[TR_PREFETCHED] = ptx::globaltimer();
-    if (!ptx::mbar_wait(rbar, 0, a.timeout_ns)) atomicOr(a.status, RTV_DEV_TIMEOUT);
+    if (cs > 1 && !ptx::mbar_wait(rbar, 0, a.timeout_ns)) atomicOr(a.status, RTV_DEV_TIMEOUT);
     if (trace && tid == 0) trace[TR_RECV] = ptx::globaltimer();
     // My incoming copies are complete (seen on rbar), so the copies that read
     // the senders' shared memory are done too; the arrive needs no ordering.
