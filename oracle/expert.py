@@ -51,6 +51,21 @@ Where the pages are silent the plainest reading is taken:
      codes with one fp32 scale per output row; W = decode(code) * scale,
      everything else unchanged (bf16 activations, fp32 accumulation on the
      device; fp64 here).
+  R16 Pi0 time conditioning (the pi0-concat workload; the "VLA design space"
+     slides and [DM0.5] 5.2 name the time MLP without its form): an action
+     token is W_to . swish(W_ti . [W_ai x + b_ai ; e(t)] + b_ti) + b_to, with
+     e(t) of the model width as in R2 and W_ti of shape [w][2w]; nothing is
+     added to it afterwards; the state token is unchanged.
+  R17 DM0.5 per-layer time modulator ([DM0.5] 5.2 lists a time modulator in
+     every layer and no formula; the dm05-adarms workload): the adaptive
+     norm of the adaLN-Zero form (Peebles and Xie, "Scalable Diffusion
+     Models with Transformers"): c(t) as in R2; per layer
+     m = time_mod.w . c + time_mod.b, split into (scale_a, shift_a, gate_a,
+     scale_m, shift_m, gate_m); each norm becomes
+     x / rms(x) * (1 + scale) + shift on every suffix row and each branch's
+     output is multiplied by its gate before the residual add; the final
+     norm stays plain; c is not added to the tokens.  6 w^2 + 6 w
+     parameters per layer (113M at width 1024 over 18 layers).
   R9 verify: per-row L2 distance over all action dims, strict d < delta,
      accepted length = longest prefix passing at every tau, one eps shared by
      all taus, gripper switch = sign (value > 0) change between consecutive
@@ -148,6 +163,19 @@ def time_condition(W: Dict[str, np.ndarray], t: float) -> np.ndarray:
     return linear(swish(z), W["time_mlp_out.w"], W["time_mlp_out.b"])
 
 
+def time_mlp_concat(W: Dict[str, np.ndarray], a: np.ndarray, t: float) -> np.ndarray:
+    """Pi0's action-time MLP over [a ; e(t)] for action embeddings a [H][w] (reading R16)."""
+    e = np.broadcast_to(time_embedding(t, a.shape[-1]), a.shape)
+    z = linear(np.concatenate([a, e], axis=-1), W["time_mlp_in.w"], W["time_mlp_in.b"])
+    return linear(swish(z), W["time_mlp_out.w"], W["time_mlp_out.b"])
+
+
+def time_modulation(W: Dict[str, np.ndarray], l: int, c: np.ndarray):
+    """Layer l's (scale_a, shift_a, gate_a, scale_m, shift_m, gate_m) from c(t) (reading R17)."""
+    m = linear(c, W[f"layers.{l}.time_mod.w"], W[f"layers.{l}.time_mod.b"])
+    return np.split(m, 6, axis=-1)
+
+
 def rope(x: np.ndarray, positions: np.ndarray, theta: float) -> np.ndarray:
     """Rotary position embedding of x [S][heads][D] (reading R4).
 
@@ -212,17 +240,32 @@ def expert_velocity(W: Dict[str, np.ndarray], cfg, x_t: np.ndarray, state: np.nd
     hq, hkv, d = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim
     eps = cfg.rms_eps
 
-    # suffix embedding: state token, then action tokens + time condition
-    c = time_condition(W, t)
+    # suffix embedding: state token, then action tokens with the time
+    # condition (added, R2; through Pi0's concat MLP, R16; or, R17, only
+    # through the per-layer modulator)
+    tc = getattr(cfg, "time_cond", "add")
     h = np.empty((s_len, cfg.width), dtype=F64)
     h[0] = linear(np.asarray(state, F64), W["state_proj.w"], W["state_proj.b"])
-    h[1:] = linear(np.asarray(x_t, F64), W["action_in_proj.w"], W["action_in_proj.b"]) + c
+    a = linear(np.asarray(x_t, F64), W["action_in_proj.w"], W["action_in_proj.b"])
+    c = time_condition(W, t) if tc != "concat" else None
+    if tc == "add":
+        h[1:] = a + c
+    elif tc == "concat":
+        h[1:] = time_mlp_concat(W, a, t)
+    elif tc == "adarms":
+        h[1:] = a
+    else:
+        raise ValueError(tc)
 
     positions = p_len + np.arange(s_len)
     visible = suffix_visibility(s_len, p_len, cfg.suffix_mask)
     for l in range(cfg.n_layers):
         p = f"layers.{l}."
-        u = rms_norm(h, W[p + "attn_norm.g"], eps)
+        if tc == "adarms":
+            sa, ba, ga, sm, bm, gm = time_modulation(W, l, c)
+            u = rms_norm(h, sa, eps) + ba
+        else:
+            u = rms_norm(h, W[p + "attn_norm.g"], eps)
         q = linear(u, W[p + "q_proj.w"]).reshape(s_len, hq, d)
         k = linear(u, W[p + "k_proj.w"]).reshape(s_len, hkv, d)
         v = linear(u, W[p + "v_proj.w"]).reshape(s_len, hkv, d)
@@ -231,10 +274,14 @@ def expert_velocity(W: Dict[str, np.ndarray], cfg, x_t: np.ndarray, state: np.nd
         keys = np.concatenate([prefix_k[l].astype(F64), k], axis=0)
         vals = np.concatenate([prefix_v[l].astype(F64), v], axis=0)
         o = attention(q, keys, vals, visible).reshape(s_len, hq * d)
-        h = h + linear(o, W[p + "o_proj.w"])
-        u = rms_norm(h, W[p + "mlp_norm.g"], eps)
+        if tc == "adarms":
+            h = h + ga * linear(o, W[p + "o_proj.w"])
+            u = rms_norm(h, sm, eps) + bm
+        else:
+            h = h + linear(o, W[p + "o_proj.w"])
+            u = rms_norm(h, W[p + "mlp_norm.g"], eps)
         m = gelu_tanh(linear(u, W[p + "gate_proj.w"])) * linear(u, W[p + "up_proj.w"])
-        h = h + linear(m, W[p + "down_proj.w"])
+        h = h + (gm if tc == "adarms" else 1.0) * linear(m, W[p + "down_proj.w"])
 
     hf = rms_norm(h[1:], W["final_norm.g"], eps)
     return linear(hf, W["action_out_proj.w"], W["action_out_proj.b"])

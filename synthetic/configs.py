@@ -15,6 +15,10 @@ Names:
                  + 48 text), 1 state token + 50 action tokens of dim 32.
   pi0-verify     FLASH verification on the pi0-bf16 expert, taus 0.2/0.5/0.8.
   pi0-fp8mlp     pi0-bf16 with FP8 E4M3 MLP weights and a 560-token prefix.
+  pi0-concat     pi0-bf16 with Pi0's time conditioning: the time MLP reads the
+                 action embedding concatenated with e(t).
+  dm05-adarms    pi0-bf16 with DM0.5's per-layer time modulator (scale, shift
+                 and gate of each norm's branch from c(t)).
 
 Draft models ("Realtime-VLA FLASH" sec. 03.1: one Gemma block and a linear
 action head, about 110M parameters, learnable action queries reading the
@@ -57,6 +61,11 @@ class ExpertShape:
     dtype: str = "f32"      # storage/MMA type of matrices and prefix KV: "f32" | "bf16"
     mlp_dtype: str = "same"  # "same" | "fp8_e4m3"
     suffix_mask: str = "bidir"  # "bidir" | "pi0_block"
+    # how the flow time enters the expert: "add" (c(t) added to the action
+    # tokens), "concat" (Pi0: time MLP over [action embedding ; e(t)]),
+    # "adarms" (DM0.5: a per-layer time modulator scaling, shifting and gating
+    # each norm's branch)
+    time_cond: str = "add"
     rms_eps: float = 1e-6
     rope_theta: float = 10000.0
     weight_std: float = 0.02
@@ -90,7 +99,10 @@ class ExpertShape:
 
     def layer_params(self) -> int:
         w, f = self.width, self.mlp_dim
-        return self.n_layers * (w * (self.q_dim + 2 * self.kv_dim) + self.q_dim * w + 3 * w * f)
+        per = w * (self.q_dim + 2 * self.kv_dim) + self.q_dim * w + 3 * w * f
+        if self.time_cond == "adarms":
+            per += 6 * w * w
+        return self.n_layers * per
 
 
 TINY_FP32 = ExpertShape(
@@ -109,7 +121,10 @@ PI0_VERIFY = PI0_BF16.with_(name="pi0-verify")
 
 PI0_FP8MLP = PI0_BF16.with_(name="pi0-fp8mlp", mlp_dtype="fp8_e4m3", prefix_len=560)
 
-CONFIGS = {c.name: c for c in (TINY_FP32, PI0_BF16, PI0_VERIFY, PI0_FP8MLP)}
+PI0_CONCAT = PI0_BF16.with_(name="pi0-concat", time_cond="concat")
+DM05_ADARMS = PI0_BF16.with_(name="dm05-adarms", time_cond="adarms")
+
+CONFIGS = {c.name: c for c in (TINY_FP32, PI0_BF16, PI0_VERIFY, PI0_FP8MLP, PI0_CONCAT, DM05_ADARMS)}
 
 
 @dataclass(frozen=True)

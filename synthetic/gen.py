@@ -94,21 +94,26 @@ def e4m3_encode(x: np.ndarray) -> np.ndarray:
 def weight_names(cfg: ExpertShape) -> List[Tuple[str, Tuple[int, ...]]]:
     """(name, shape) of every expert parameter, matrices as [out][in]."""
     w, a, sd, f = cfg.width, cfg.action_dim, cfg.state_dim, cfg.mlp_dim
+    tin = 2 * w if cfg.time_cond == "concat" else w
     out = [
         ("state_proj.w", (w, sd)), ("state_proj.b", (w,)),
         ("action_in_proj.w", (w, a)), ("action_in_proj.b", (w,)),
-        ("time_mlp_in.w", (w, w)), ("time_mlp_in.b", (w,)),
+        ("time_mlp_in.w", (w, tin)), ("time_mlp_in.b", (w,)),
         ("time_mlp_out.w", (w, w)), ("time_mlp_out.b", (w,)),
     ]
+    adarms = cfg.time_cond == "adarms"
     for l in range(cfg.n_layers):
         p = f"layers.{l}."
+        out += [] if adarms else [(p + "attn_norm.g", (w,))]
         out += [
-            (p + "attn_norm.g", (w,)),
             (p + "q_proj.w", (cfg.q_dim, w)),
             (p + "k_proj.w", (cfg.kv_dim, w)),
             (p + "v_proj.w", (cfg.kv_dim, w)),
             (p + "o_proj.w", (w, cfg.q_dim)),
-            (p + "mlp_norm.g", (w,)),
+        ]
+        out += [(p + "time_mod.w", (6 * w, w)), (p + "time_mod.b", (6 * w,))] if adarms else \
+            [(p + "mlp_norm.g", (w,))]
+        out += [
             (p + "gate_proj.w", (f, w)),
             (p + "up_proj.w", (f, w)),
             (p + "down_proj.w", (w, f)),

@@ -57,10 +57,25 @@ def velocity(W, cfg, x_t, state, t, prefix_k, prefix_v):
     w = cfg.width
     eps = cfg.rms_eps
 
+    tc = getattr(cfg, "time_cond", "add")
     st = F.linear(_t(state), _t(W["state_proj.w"]), _t(W["state_proj.b"]))
     act = F.linear(x_t, _t(W["action_in_proj.w"]), _t(W["action_in_proj.b"]))
-    c = torch.stack([time_cond(W, float(tt), w) for tt in t])      # [G, w]
-    h = torch.cat([st.expand(g_count, 1, w), act + c[:, None, :]], dim=1)  # [G, S, w]
+    if tc == "concat":
+        emb = []
+        for g in range(g_count):
+            half = w // 2
+            expo = torch.linspace(0.0, 1.0, half, dtype=T64)
+            period = 4e-3 * torch.pow(torch.tensor(4.0 / 4e-3, dtype=T64), expo)
+            ang = 2 * math.pi * float(t[g]) / period
+            e = torch.cat([torch.sin(ang), torch.cos(ang)]).expand(h_len, w)
+            z = F.linear(torch.cat([act[g], e], dim=-1), _t(W["time_mlp_in.w"]), _t(W["time_mlp_in.b"]))
+            emb.append(F.linear(F.silu(z), _t(W["time_mlp_out.w"]), _t(W["time_mlp_out.b"])))
+        tokens = torch.stack(emb)
+        c = None
+    else:
+        c = torch.stack([time_cond(W, float(tt), w) for tt in t])      # [G, w]
+        tokens = act + c[:, None, :] if tc == "add" else act
+    h = torch.cat([st.expand(g_count, 1, w), tokens], dim=1)  # [G, S, w]
 
     pos = torch.arange(p_len, p_len + s_len)
     mask = torch.ones(s_len, p_len + s_len, dtype=torch.bool)
@@ -69,7 +84,12 @@ def velocity(W, cfg, x_t, state, t, prefix_k, prefix_v):
 
     for l in range(cfg.n_layers):
         p = f"layers.{l}."
-        u = F.rms_norm(h, (w,), weight=1.0 + _t(W[p + "attn_norm.g"]), eps=eps)
+        if tc == "adarms":
+            mod = F.linear(c, _t(W[p + "time_mod.w"]), _t(W[p + "time_mod.b"]))[:, None, :]   # [G, 1, 6w]
+            sa, ba, ga, sm, bm, gm = torch.chunk(mod, 6, dim=-1)
+            u = F.rms_norm(h, (w,), eps=eps) * (1.0 + sa) + ba
+        else:
+            u = F.rms_norm(h, (w,), weight=1.0 + _t(W[p + "attn_norm.g"]), eps=eps)
         q = F.linear(u, _t(W[p + "q_proj.w"])).view(g_count, s_len, hq, d)
         k = F.linear(u, _t(W[p + "k_proj.w"])).view(g_count, s_len, hkv, d)
         v = F.linear(u, _t(W[p + "v_proj.w"])).view(g_count, s_len, hkv, d)
@@ -84,10 +104,15 @@ def velocity(W, cfg, x_t, state, t, prefix_k, prefix_v):
         vals = vals.repeat_interleave(rep, dim=1)
         o = F.scaled_dot_product_attention(q.transpose(1, 2), keys, vals, attn_mask=mask)
         o = o.transpose(1, 2).reshape(g_count, s_len, hq * d)
-        h = h + F.linear(o, _t(W[p + "o_proj.w"]))
-        u = F.rms_norm(h, (w,), weight=1.0 + _t(W[p + "mlp_norm.g"]), eps=eps)
+        if tc == "adarms":
+            h = h + ga * F.linear(o, _t(W[p + "o_proj.w"]))
+            u = F.rms_norm(h, (w,), eps=eps) * (1.0 + sm) + bm
+        else:
+            h = h + F.linear(o, _t(W[p + "o_proj.w"]))
+            u = F.rms_norm(h, (w,), weight=1.0 + _t(W[p + "mlp_norm.g"]), eps=eps)
         gate = F.gelu(F.linear(u, _t(W[p + "gate_proj.w"])), approximate="tanh")
-        h = h + F.linear(gate * F.linear(u, _t(W[p + "up_proj.w"])), _t(W[p + "down_proj.w"]))
+        branch = F.linear(gate * F.linear(u, _t(W[p + "up_proj.w"])), _t(W[p + "down_proj.w"]))
+        h = h + (gm * branch if tc == "adarms" else branch)
 
     hf = F.rms_norm(h[:, 1:], (w,), weight=1.0 + _t(W["final_norm.g"]), eps=eps)
     return F.linear(hf, _t(W["action_out_proj.w"]), _t(W["action_out_proj.b"])).numpy()
