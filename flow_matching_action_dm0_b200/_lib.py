@@ -20,6 +20,7 @@ STATUS_NAMES = ["RTV_OK", "RTV_ERR_ARG", "RTV_ERR_SHAPE", "RTV_ERR_STATE", "RTV_
                 "RTV_ERR_TIMEOUT", "RTV_ERR_NUMERIC", "RTV_ERR_UNSUPPORTED"]
 RTV_F32, RTV_BF16, RTV_FP8_E4M3, RTV_SAME = 0, 1, 2, 3
 RTV_MASK_BIDIR, RTV_MASK_PI0_BLOCK = 0, 1
+RTV_TIME_ADD, RTV_TIME_CONCAT, RTV_TIME_ADARMS = 0, 1, 2
 RTV_DEV_TIMEOUT, RTV_DEV_NUMERIC, RTV_DEV_BOUNDS = 1, 2, 4
 RTV_FLAG_ZERO_ACCEPT, RTV_FLAG_SWITCH, RTV_FLAG_SWITCH_IN_PREFIX = 1, 2, 4
 
@@ -39,6 +40,7 @@ class rtv_expert_config(C.Structure):
         ("chunk_len", C.c_int), ("max_prefix_len", C.c_int), ("max_batch", C.c_int), ("max_taus", C.c_int),
         ("dtype", C.c_int), ("mlp_dtype", C.c_int), ("suffix_mask", C.c_int),
         ("rms_eps", C.c_float), ("rope_theta", C.c_float), ("barrier_timeout_ns", C.c_longlong),
+        ("time_cond", C.c_int),
     ]
 
 

@@ -10,6 +10,8 @@ struct rtv_ctx;
 
 namespace rtv {
 
+struct ModTables;
+
 // Decide whether the config can use the tensor-core path and allocate its
 // state; sets ctx->use_fast.  Returns an error only on a CUDA failure.
 rtv_status fast_create(rtv_ctx* ctx);
@@ -21,11 +23,17 @@ rtv_status fast_prefix_update(rtv_ctx* ctx, int batch, int prefix_len, cudaStrea
 // Step boundary over G suffixes: output head (Euler update of ctx->x, or the
 // velocity into ctx->v when velocity_only) and/or the suffix embedding of the
 // next evaluation into ctx->h with time condition rows c (stride c_stride).
+// g0 (group stride g0_stride), when set, replaces the first layer's
+// attention-norm gain in the embedding's norm input.
 rtv_status fast_step(rtv_ctx* ctx, int G, bool do_head, bool do_embed, float dt, const float* c, int c_stride,
-                     int state_stride, bool velocity_only, cudaStream_t st);
-// The expert's layers over G suffixes (residual stream ctx->h).
+                     int state_stride, bool velocity_only, cudaStream_t st, const float* g0 = nullptr,
+                     int g0_stride = 0);
+// The expert's layers over G suffixes (residual stream ctx->h); mod set for
+// RTV_TIME_ADARMS.
 rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, const float* rope_cs,
-                       const float* rope_sn, cudaStream_t st);
+                       const float* rope_sn, cudaStream_t st, const ModTables* mod = nullptr);
+// The first layer's norm input of the residual rows of G suffixes, from ctx->h.
+rtv_status fast_norm_rows(rtv_ctx* ctx, int G, cudaStream_t st);
 // Bare block (ctx->block_only), layer 0: keys and values of n_vis tokens per
 // batch element given as bf16 rows vis [batch][n_vis][width] (RMSNorm, K/V
 // projection, RoPE at positions 0..n_vis-1), written into the cached prefix,

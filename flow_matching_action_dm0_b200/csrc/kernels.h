@@ -33,6 +33,19 @@ void launch_attention_simt(const float* q, const KT* pk, const KT* pv, const flo
 
 void launch_geglu(const float* gu, float* m, int T, int F, cudaStream_t st);
 
+// y[t][n] = act(x[t] . W[n] + bias[t / S][n]) (EPI_ADD: +=) for rows t < T
+// with t % S in [s_lo, s_hi); W rows of stride ldw; bias group stride bias_gs.
+template <typename WT>
+void launch_rows_linear(const float* x, int ldx, const WT* W, int ldw, const float* bias, int bias_gs, float* y,
+                        int ldy, int T, int S, int s_lo, int s_hi, int N, int K, int epi, cudaStream_t st);
+
+// u = h / rms(h) * (1 + scale[t / S]) + shift[t / S] (group stride gs).
+void launch_rmsnorm_mod(const float* h, const float* scale, const float* shift, int gs, float* u, int rows, int w,
+                        int S, float eps, cudaStream_t st);
+
+// h[t] += gate[t / S] * b[t] (group stride gs).
+void launch_gated_add(float* h, const float* b, const float* gate, int gs, int w, int S, int T, cudaStream_t st);
+
 template <typename WT>
 void launch_out_head(const float* h, const float* gain, const WT* w_ao, const float* b_ao, float* x, float* vout,
                      float dt, int G, int w, int S, int A, float eps, unsigned* status, cudaStream_t st);

@@ -5,6 +5,8 @@
 // verification decision).
 #include <math.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -399,6 +401,109 @@ __global__ void prefix_pack_kernel(const KT* __restrict__ src, KT* __restrict__ 
 // ---------------------------------------------------------------------------
 // host launchers
 // ---------------------------------------------------------------------------
+// ---------------------------------------------------------------------------
+// Linear map of a few rows with a per-group bias, for the time-conditioning
+// variants: y[t][n] = act(sum_k x[t][k] W[n][k] + bias[g][n]) (EPI_ADD adds
+// into y) for the rows t < T whose position s = t % S lies in [s_lo, s_hi),
+// g = t / S; W rows have stride ldw.  A CTA takes 8 outputs (a warp each)
+// and 32 rows staged in shared memory 256 inputs at a time; a lane reads 8
+// consecutive weights per step (K and ldw multiples of 8).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void load8w(const float* p, float v[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void load8w(const __nv_bfloat16* p, float v[8]) {
+  const uint4 q = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h2[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
+template <typename WT, int EPI>
+__global__ void __launch_bounds__(256) rows_linear_kernel(const float* __restrict__ x, int ldx,
+                                                          const WT* __restrict__ W, int ldw,
+                                                          const float* __restrict__ bias, int bias_gs,
+                                                          float* __restrict__ y, int ldy, int T, int S, int s_lo,
+                                                          int s_hi, int N, int K) {
+  __shared__ float xs[32][260];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = blockIdx.x * 8 + warp;
+  const int r0 = blockIdx.y * 32;
+  float acc[32];
+#pragma unroll
+  for (int r = 0; r < 32; ++r) acc[r] = 0.f;
+  for (int k0 = 0; k0 < K; k0 += 256) {
+    const int kc = min(256, K - k0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < 32 * 256; i += 256) {
+      const int r = i >> 8, kk = i & 255;
+      xs[r][kk] = (r0 + r < T && kk < kc) ? x[(size_t)(r0 + r) * ldx + k0 + kk] : 0.f;
+    }
+    __syncthreads();
+    if (n < N && lane * 8 < kc) {
+      float wv[8];
+      load8w(W + (size_t)n * ldw + k0 + lane * 8, wv);
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        float v = acc[r];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v = fmaf(xs[r][lane * 8 + e], wv[e], v);
+        acc[r] = v;
+      }
+    }
+  }
+  if (n >= N) return;
+#pragma unroll
+  for (int r = 0; r < 32; ++r) {
+    float v = warp_sum(acc[r]);
+    const int t = r0 + r;
+    if (lane == 0 && t < T) {
+      const int g = t / S, sp = t - g * S;
+      if (sp >= s_lo && sp < s_hi) {
+        if (bias) v += bias[(size_t)g * bias_gs + n];
+        float* yp = y + (size_t)t * ldy + n;
+        if (EPI == EPI_ADD) *yp += v;
+        else if (EPI == EPI_SWISH) *yp = swish(v);
+        else *yp = v;
+      }
+    }
+  }
+}
+
+// Modulated RMSNorm of the per-layer time modulator: u = h / rms(h) * (1 +
+// scale[g]) + shift[g] for row t of group g = t / S.
+__global__ void rmsnorm_mod_kernel(const float* __restrict__ h, const float* __restrict__ scale,
+                                   const float* __restrict__ shift, int gs, float* __restrict__ u, int w, int S,
+                                   float eps) {
+  __shared__ float red[32];
+  const int t = blockIdx.x, g = t / S;
+  const float* row = h + (size_t)t * w;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < w; i += blockDim.x) ss = fmaf(row[i], row[i], ss);
+  ss = block_sum(ss, red);
+  const float inv = rsqrtf(ss / (float)w + eps);
+  const float* sc = scale + (size_t)g * gs;
+  const float* sh = shift + (size_t)g * gs;
+  for (int i = threadIdx.x; i < w; i += blockDim.x) u[(size_t)t * w + i] = row[i] * inv * (1.f + sc[i]) + sh[i];
+}
+
+// Gated residual add: h[t] += gate[g] * b[t], g = t / S.
+__global__ void gated_add_kernel(float* __restrict__ h, const float* __restrict__ b, const float* __restrict__ gate,
+                                 int gs, int w, int S, int T) {
+  const size_t n = (size_t)T * w;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const size_t t = i / w, k = i % w;
+    h[i] += gate[(t / S) * (size_t)gs + k] * b[i];
+  }
+}
+
 void launch_time_embedding(const float* taus, int n, int n_steps, float* e, int w, cudaStream_t st) {
   time_embedding_kernel<<<n, 128, 0, st>>>(taus, n_steps, e, w);
 }
@@ -497,5 +602,35 @@ void launch_prefix_pack(const KT* src, KT* dst, int L, int B, int P, int Hkv, in
 template void launch_prefix_pack<float>(const float*, float*, int, int, int, int, int, int, int, cudaStream_t);
 template void launch_prefix_pack<__nv_bfloat16>(const __nv_bfloat16*, __nv_bfloat16*, int, int, int, int, int, int,
                                                 int, cudaStream_t);
+
+template <typename WT>
+void launch_rows_linear(const float* x, int ldx, const WT* W, int ldw, const float* bias, int bias_gs, float* y,
+                        int ldy, int T, int S, int s_lo, int s_hi, int N, int K, int epi, cudaStream_t st) {
+  dim3 grid((N + 7) / 8, (T + 31) / 32);
+  if (epi == EPI_ADD)
+    rows_linear_kernel<WT, EPI_ADD><<<grid, 256, 0, st>>>(x, ldx, W, ldw, bias, bias_gs, y, ldy, T, S, s_lo, s_hi,
+                                                          N, K);
+  else if (epi == EPI_SWISH)
+    rows_linear_kernel<WT, EPI_SWISH><<<grid, 256, 0, st>>>(x, ldx, W, ldw, bias, bias_gs, y, ldy, T, S, s_lo,
+                                                            s_hi, N, K);
+  else
+    rows_linear_kernel<WT, EPI_STORE><<<grid, 256, 0, st>>>(x, ldx, W, ldw, bias, bias_gs, y, ldy, T, S, s_lo,
+                                                            s_hi, N, K);
+}
+template void launch_rows_linear<float>(const float*, int, const float*, int, const float*, int, float*, int, int,
+                                        int, int, int, int, int, int, cudaStream_t);
+template void launch_rows_linear<__nv_bfloat16>(const float*, int, const __nv_bfloat16*, int, const float*, int,
+                                                float*, int, int, int, int, int, int, int, int, cudaStream_t);
+
+void launch_rmsnorm_mod(const float* h, const float* scale, const float* shift, int gs, float* u, int rows, int w,
+                        int S, float eps, cudaStream_t st) {
+  rmsnorm_mod_kernel<<<rows, 256, 0, st>>>(h, scale, shift, gs, u, w, S, eps);
+}
+
+void launch_gated_add(float* h, const float* b, const float* gate, int gs, int w, int S, int T, cudaStream_t st) {
+  const size_t n = (size_t)T * w;
+  const int blocks = (int)std::min<size_t>((n + 255) / 256, 4096);
+  gated_add_kernel<<<blocks, 256, 0, st>>>(h, b, gate, gs, w, S, T);
+}
 
 }  // namespace rtv

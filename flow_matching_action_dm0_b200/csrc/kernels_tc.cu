@@ -119,6 +119,12 @@ struct GemmArgs {
   int seq;                    // QKV: tokens of one sequence -- RoPE position and ks/vs row are t % seq, the
                               // sequence t / seq (= S for suffixes; the prefix length for a prefix)
   int kv_prefix;              // QKV with qt set: keys and values still go to ks / vs rows, not to kts / vts
+  // Per-layer time modulator (each suffix group g = t / S reads its own row):
+  int g_stride;               // O, DOWN: the next norm's gain is g_next + g * g_stride (0: one gain for all)
+  const float* sb;            // QKV, GU: added after the 1/rms factor, sb[g * sb_stride + natural row]
+  int sb_stride;
+  const float* gate;          // O, DOWN: the branch is multiplied by gate[g * gate_stride + feature]
+  int gate_stride;
   float eps;
 };
 
@@ -477,6 +483,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
 #pragma unroll 1
     for (int tl = ew; tl < n_own; tl += kEpiWarps) {
       const int t = t0 + t_own0 + tl;   // global token row
+      const int tg = t / a.S;           // its suffix group
       float2 x1 = make_float2(0.f, 0.f), x2 = make_float2(0.f, 0.f);
       for (int qr = 0; qr < cs; ++qr) {
         const float* rr = recv + (qr * per + tl) * 128;
@@ -492,6 +499,19 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
         x1.y *= ws1.y;
         x2.x *= ws2.x;
         x2.y *= ws2.y;
+      }
+      if ((MODE == GM_O || MODE == GM_DOWN) && a.gate) {   // gated branch (time modulator)
+        const float* gp = a.gate + (size_t)tg * a.gate_stride;
+        const float2 q1 = *reinterpret_cast<const float2*>(gp + n1);
+        const float2 q2 = *reinterpret_cast<const float2*>(gp + n2);
+        x1.x *= q1.x;
+        x1.y *= q1.y;
+        x2.x *= q2.x;
+        x2.y *= q2.y;
+      }
+      if ((MODE == GM_O || MODE == GM_DOWN) && a.g_next && a.g_stride) {   // per-group gain of the next norm
+        gn1 = *reinterpret_cast<const float2*>(a.g_next + (size_t)tg * a.g_stride + n1);
+        gn2 = *reinterpret_cast<const float2*>(a.g_next + (size_t)tg * a.g_stride + n2);
       }
       if (MODE == GM_O || MODE == GM_DOWN) {
         // residual add, then the next norm's bf16 input and this tile's sum of squares
@@ -519,6 +539,15 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
         x1.y *= rs;
         x2.x *= rs;
         x2.y *= rs;
+        if (a.sb) {   // the modulator's shift carried through the projection (natural row order)
+          const float* sp = a.sb + (size_t)tg * a.sb_stride;
+          const int r1 = MODE == GM_GU ? 64 * nt + f0 : hh * a.D + dq0 + f0;
+          const int r2 = MODE == GM_GU ? a.F + 64 * nt + f0 : hh * a.D + dq0 + hd + f0;
+          x1.x += sp[r1];
+          x1.y += sp[r1 + 1];
+          x2.x += sp[r2];
+          x2.y += sp[r2 + 1];
+        }
         if (MODE == GM_GU) {
           *reinterpret_cast<uint32_t*>(a.m + ts_offset(t, nt * 64 + f0, n_rows)) =
               ptx::pack_bf16x2(gelu_tanh(x1.x) * x2.x, gelu_tanh(x1.y) * x2.y);
@@ -1218,9 +1247,9 @@ struct StepArgs {
   const float* b_ai;
   const __nv_bfloat16* w_spT;     // [Sd][w] (state_proj transposed)
   const float* b_sp;
-  const float* g_attn0;           // first layer's attention-norm gain
+  const float* g_attn0;           // first layer's attention-norm gain (of group g: g_attn0 + g * g0_stride)
   unsigned* status;
-  int w, S, A, Sd, state_stride, c_stride, do_head, do_embed, n_mma;
+  int w, S, A, Sd, state_stride, c_stride, do_head, do_embed, n_mma, g0_stride;
   float dt, eps;
 };
 
@@ -1316,7 +1345,7 @@ __global__ void __launch_bounds__(256) step_kernel(const StepArgs a) {
     if (s > 0) hv[e] += a.c[(size_t)g * a.c_stride + i0 + e];
   }
   *reinterpret_cast<float4*>(a.h + (size_t)r * a.w + i0) = make_float4(hv[0], hv[1], hv[2], hv[3]);
-  const float4 ga = *reinterpret_cast<const float4*>(a.g_attn0 + i0);
+  const float4 ga = *reinterpret_cast<const float4*>(a.g_attn0 + (size_t)g * a.g0_stride + i0);
   uint2 hbv;
   hbv.x = ptx::pack_bf16x2(hv[0] * (1.f + ga.x), hv[1] * (1.f + ga.y));
   hbv.y = ptx::pack_bf16x2(hv[2] * (1.f + ga.z), hv[3] * (1.f + ga.w));
@@ -1909,7 +1938,7 @@ rtv_status fast_load(rtv_ctx* ctx, const rtv_tensor*, int) {
 }
 
 rtv_status fast_step(rtv_ctx* ctx, int G, bool do_head, bool do_embed, float dt, const float* c, int c_stride,
-                     int state_stride, bool velocity_only, cudaStream_t st) {
+                     int state_stride, bool velocity_only, cudaStream_t st, const float* g0, int g0_stride) {
   FastPath* fp = ctx->fast;
   const rtv_expert_config& k = ctx->cfg;
   StepArgs a{};
@@ -1927,7 +1956,8 @@ rtv_status fast_step(rtv_ctx* ctx, int G, bool do_head, bool do_embed, float dt,
   a.b_ai = ctx->W.ai_b;
   a.w_spT = fp->w_spT;
   a.b_sp = ctx->W.sp_b;
-  a.g_attn0 = ctx->W.layers[0].g_attn;
+  a.g_attn0 = g0 ? g0 : ctx->W.layers[0].g_attn;
+  a.g0_stride = g0 ? g0_stride : 0;
   a.status = ctx->status;
   a.w = k.width;
   a.S = ctx->S;
@@ -2178,8 +2208,21 @@ rtv_status fast_prefill(rtv_ctx* pre, rtv_ctx* ex, const __nv_bfloat16* emb, int
   return RTV_OK;
 }
 
+rtv_status fast_norm_rows(rtv_ctx* ctx, int G, cudaStream_t st) {
+  FastPath* fp = ctx->fast;
+  const int T = G * ctx->S;
+  norm_input_kernel<float><<<T, 128, 0, st>>>(ctx->h, T, nullptr, ctx->W.layers[0].g_attn, fp->hb, fp->ssp,
+                                              round_up(T, 16), ctx->cfg.width);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    ctx->last_error = std::string("norm input launch: ") + cudaGetErrorString(e);
+    return RTV_ERR_CUDA;
+  }
+  return RTV_OK;
+}
+
 rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, const float* rope_cs,
-                       const float* rope_sn, cudaStream_t st) {
+                       const float* rope_sn, cudaStream_t st, const ModTables* mod) {
   FastPath* fp = ctx->fast;
   const rtv_expert_config& k = ctx->cfg;
   const int S = ctx->S, T = G * S, w = k.width, F = k.mlp_dim, D = k.head_dim, Q = ctx->Q, KV = ctx->KV;
@@ -2302,10 +2345,18 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     return (tracing && l == 0) ? fp->trace + (size_t)i * 512 * kTraceRow : nullptr;
   };
 
+  // per-layer time modulator rows (RTV_TIME_ADARMS): group strides
+  const int L6 = k.n_layers * 6 * w;
+  const int mg = mod ? mod->group_rows : 0;
   for (int l = 0; l < k.n_layers; ++l) {
     const LayerW& Lw = ctx->W.layers[l];
+    const float* ml = mod ? mod->mod + (size_t)l * 6 * w : nullptr;
     GemmArgs a = base;
     a.trace = tr(l, 0);
+    if (mod) {
+      a.sb = mod->sbq + (size_t)l * nq;
+      a.sb_stride = mg * k.n_layers * nq;
+    }
     a.wt = fp->w_qkv;
     a.act = fp->hb;
     a.K = w;
@@ -2336,6 +2387,12 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     a.pf = fp->mlp_f8 ? fp->w_gu8 + (size_t)l * 2 * F * w : (const uint8_t*)(fp->w_gu + (size_t)l * 2 * F * w);
     a.pf_bytes = (unsigned long long)2 * F * w * (fp->mlp_f8 ? 1 : 2);
     a.g_next = Lw.g_mlp;
+    if (mod) {
+      a.gate = ml + 2 * w;
+      a.gate_stride = mg * L6;
+      a.g_next = ml + 3 * w;
+      a.g_stride = mg * L6;
+    }
     if (e == cudaSuccess) e = launch_gemm<GM_O>(a, p_o, st, fp->pf_cap);
 
     a = base;
@@ -2348,6 +2405,10 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     a.w_tile0 = l * 2 * F / 128;
     a.pf = fp->mlp_f8 ? fp->w_down8 + (size_t)l * w * F : (const uint8_t*)(fp->w_down + (size_t)l * w * F);
     a.pf_bytes = (unsigned long long)w * F * (fp->mlp_f8 ? 1 : 2);
+    if (mod) {
+      a.sb = mod->sbg + (size_t)l * 2 * F;
+      a.sb_stride = mg * k.n_layers * 2 * F;
+    }
     if (e == cudaSuccess) e = launch_gemm<GM_GU>(a, p_gu, st, fp->pf_cap);
 
     a = base;
@@ -2361,6 +2422,12 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     a.pf = (const uint8_t*)(fp->w_qkv + (size_t)((l + 1) % k.n_layers) * nq * w);
     a.pf_bytes = (unsigned long long)nq * w * 2;
     a.g_next = (l + 1 < k.n_layers) ? ctx->W.layers[l + 1].g_attn : nullptr;
+    if (mod) {
+      a.gate = ml + 5 * w;
+      a.gate_stride = mg * L6;
+      a.g_next = (l + 1 < k.n_layers) ? ml + 6 * w : nullptr;   // scale_a of the next layer
+      a.g_stride = mg * L6;
+    }
     if (e == cudaSuccess) e = launch_gemm<GM_DOWN>(a, p_dn, st, fp->pf_cap);
     if (e != cudaSuccess) {
       ctx->last_error = std::string("tensor-core launch: ") + cudaGetErrorString(e);

@@ -26,29 +26,76 @@ namespace rtv {
 // residual.
 template <typename WT>
 void simt_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, const float* rope_cs, const float* rope_sn,
-                 cudaStream_t st) {
+                 cudaStream_t st, const ModTables* mod) {
   const rtv_expert_config& k = ctx->cfg;
   const int S = ctx->S, T = G * S, w = k.width, F = k.mlp_dim;
   const int Q = ctx->Q, KV = ctx->KV, D = k.head_dim;
   const size_t kv_layer = (size_t)k.max_batch * k.n_kv_heads * k.max_prefix_len * D;
+  const int mgs = mod ? mod->group_rows * k.n_layers * 6 * w : 0;   // group stride of the modulation rows
   for (int l = 0; l < k.n_layers; ++l) {
     const LayerW& L = ctx->W.layers[l];
     const WT* pk = (const WT*)ctx->prefix_kv + (size_t)(2 * l) * kv_layer;
     const WT* pv = (const WT*)ctx->prefix_kv + (size_t)(2 * l + 1) * kv_layer;
-    launch_rmsnorm(ctx->h, L.g_attn, ctx->u, T, w, k.rms_eps, st);
+    const float* ml = mod ? mod->mod + (size_t)l * 6 * w : nullptr;   // scale/shift/gate of the layer
+    if (ml) launch_rmsnorm_mod(ctx->h, ml, ml + w, mgs, ctx->u, T, w, S, k.rms_eps, st);
+    else launch_rmsnorm(ctx->h, L.g_attn, ctx->u, T, w, k.rms_eps, st);
     launch_linear<WT>(ctx->u, w, (const WT*)L.qkv, nullptr, ctx->qkv, Q + 2 * KV, T, Q + 2 * KV, w, EPI_STORE, st);
     launch_rope_split(ctx->qkv, rope_cs, rope_sn, ctx->q, ctx->ks, ctx->vs, T, S, k.n_q_heads, k.n_kv_heads, D, st);
     launch_attention_simt<WT>(ctx->q, pk, pv, ctx->ks, ctx->vs, ctx->o, T, S, P, k.max_prefix_len, k.n_q_heads,
                               k.n_kv_heads, D, prefix_batch_stride, k.suffix_mask, st);
-    launch_linear<WT>(ctx->o, Q, (const WT*)L.o, nullptr, ctx->h, w, T, w, Q, EPI_ADD, st);
-    launch_rmsnorm(ctx->h, L.g_mlp, ctx->u, T, w, k.rms_eps, st);
+    if (ml) {
+      launch_linear<WT>(ctx->o, Q, (const WT*)L.o, nullptr, ctx->u, w, T, w, Q, EPI_STORE, st);
+      launch_gated_add(ctx->h, ctx->u, ml + 2 * w, mgs, w, S, T, st);
+      launch_rmsnorm_mod(ctx->h, ml + 3 * w, ml + 4 * w, mgs, ctx->u, T, w, S, k.rms_eps, st);
+    } else {
+      launch_linear<WT>(ctx->o, Q, (const WT*)L.o, nullptr, ctx->h, w, T, w, Q, EPI_ADD, st);
+      launch_rmsnorm(ctx->h, L.g_mlp, ctx->u, T, w, k.rms_eps, st);
+    }
     launch_linear<WT>(ctx->u, w, (const WT*)L.gu, nullptr, ctx->gu, 2 * F, T, 2 * F, w, EPI_STORE, st);
     launch_geglu(ctx->gu, ctx->m, T, F, st);
-    launch_linear<WT>(ctx->m, F, (const WT*)L.down, nullptr, ctx->h, w, T, w, F, EPI_ADD, st);
+    if (ml) {
+      launch_linear<WT>(ctx->m, F, (const WT*)L.down, nullptr, ctx->u, w, T, w, F, EPI_STORE, st);
+      launch_gated_add(ctx->h, ctx->u, ml + 5 * w, mgs, w, S, T, st);
+    } else {
+      launch_linear<WT>(ctx->m, F, (const WT*)L.down, nullptr, ctx->h, w, T, w, F, EPI_ADD, st);
+    }
   }
 }
-template void simt_layers<float>(rtv_ctx*, int, int, int, const float*, const float*, cudaStream_t);
-template void simt_layers<__nv_bfloat16>(rtv_ctx*, int, int, int, const float*, const float*, cudaStream_t);
+template void simt_layers<float>(rtv_ctx*, int, int, int, const float*, const float*, cudaStream_t,
+                                 const ModTables*);
+template void simt_layers<__nv_bfloat16>(rtv_ctx*, int, int, int, const float*, const float*, cudaStream_t,
+                                         const ModTables*);
+
+// Pi0's concat time MLP over the action rows of G suffixes, in place in
+// ctx->h: h <- W_to swish(W_ti[:, :w] h + c1[g]) + b_to, where c1 (group
+// stride c1_gs) already holds W_ti[:, w:] e(t) + b_ti.
+template <typename WT>
+void concat_tokens(rtv_ctx* ctx, int G, const float* c1, int c1_gs, cudaStream_t st) {
+  const int w = ctx->cfg.width, S = ctx->S, T = G * S;
+  launch_rows_linear<WT>(ctx->h, w, (const WT*)ctx->W.ti_w, 2 * w, c1, c1_gs, ctx->u, w, T, S, 1, S, w, w,
+                         EPI_SWISH, st);
+  launch_rows_linear<WT>(ctx->u, w, (const WT*)ctx->W.to_w, w, ctx->W.to_b, 0, ctx->h, w, T, S, 1, S, w, w,
+                         EPI_STORE, st);
+}
+
+// Per-layer modulation rows of n flow times from their conditions c [n][w]
+// (mod), and, when sbq is set, the shifts' share of the QKV and gate/up
+// projections (sbq, sbg).
+template <typename WT>
+void mod_tables(rtv_ctx* ctx, const float* c, int n, float* mod, float* sbq, float* sbg, cudaStream_t st) {
+  const rtv_expert_config& k = ctx->cfg;
+  const int w = k.width, L = k.n_layers, nq = ctx->Q + 2 * ctx->KV, F2 = 2 * k.mlp_dim;
+  for (int l = 0; l < L; ++l) {
+    const LayerW& Lw = ctx->W.layers[l];
+    launch_rows_linear<WT>(c, w, (const WT*)Lw.tmod_w, w, Lw.tmod_b, 0, mod + (size_t)l * 6 * w, L * 6 * w, n, n, 0,
+                           n, 6 * w, w, EPI_STORE, st);
+    if (!sbq) continue;
+    launch_rows_linear<WT>(mod + (size_t)l * 6 * w + w, L * 6 * w, (const WT*)Lw.qkv, w, nullptr, 0,
+                           sbq + (size_t)l * nq, L * nq, n, n, 0, n, nq, w, EPI_STORE, st);
+    launch_rows_linear<WT>(mod + (size_t)l * 6 * w + 4 * w, L * 6 * w, (const WT*)Lw.gu, w, nullptr, 0,
+                           sbg + (size_t)l * F2, L * F2, n, n, 0, n, F2, w, EPI_STORE, st);
+  }
+}
 
 }  // namespace rtv
 
@@ -108,11 +155,13 @@ struct DeviceGuard {
 // output head.  Used for the fp32 expert and, on request, the bf16 expert.
 template <typename WT>
 void simt_expert(rtv_ctx* ctx, int G, int P, const float* c, int c_stride, int state_stride, int prefix_batch_stride,
-                 const float* rope_cs, const float* rope_sn, cudaStream_t st) {
+                 const float* rope_cs, const float* rope_sn, cudaStream_t st, const float* c1 = nullptr,
+                 int c1_gs = 0, const ModTables* mod = nullptr) {
   const rtv_expert_config& k = ctx->cfg;
   launch_embed<WT>(ctx->x, ctx->state, state_stride, (const WT*)ctx->W.sp_w, ctx->W.sp_b, (const WT*)ctx->W.ai_w,
                    ctx->W.ai_b, c, c_stride, ctx->h, G, k.width, ctx->S, k.action_dim, k.state_dim, st);
-  simt_layers<WT>(ctx, G, P, prefix_batch_stride, rope_cs, rope_sn, st);
+  if (c1) concat_tokens<WT>(ctx, G, c1, c1_gs, st);
+  simt_layers<WT>(ctx, G, P, prefix_batch_stride, rope_cs, rope_sn, st, mod);
 }
 
 // c(t) = time_mlp_out(swish(time_mlp_in(e(t)))) for n times (taus or the Euler schedule).
@@ -140,26 +189,46 @@ int count_kernel_nodes(cudaGraph_t g) {
 enum { KIND_DENOISE = 0, KIND_VERIFY = 1 };
 
 // Precompute the input-independent tables of a graph (time condition of the
-// Euler schedule, RoPE table of the suffix positions), then capture.
+// Euler schedule, RoPE table of the suffix positions, the time modulator's
+// rows), then capture.
 template <typename WT>
 rtv_status build_graph(rtv_ctx* ctx, int kind, int n, int batch, int P, GraphEntry& ge,
                        const GraphPrologue* prologue = nullptr) {
   const rtv_expert_config& k = ctx->cfg;
   cudaStream_t st = ctx->cap_stream;
-  const int S = ctx->S, D = k.head_dim, w = k.width;
-  float *cs = nullptr, *sn = nullptr, *ctab = nullptr;
-  CK(cudaMalloc(&cs, sizeof(float) * S * (D / 2)));
-  ge.owned.push_back(cs);
-  CK(cudaMalloc(&sn, sizeof(float) * S * (D / 2)));
-  ge.owned.push_back(sn);
+  const int S = ctx->S, D = k.head_dim, w = k.width, L = k.n_layers;
+  const int nq = ctx->Q + 2 * ctx->KV, F2 = 2 * k.mlp_dim;
+  const int tc = k.time_cond;
+  auto table = [&](float** p, size_t count) -> rtv_status {
+    CK(cudaMalloc(p, sizeof(float) * count));
+    ge.owned.push_back(*p);
+    return RTV_OK;
+  };
+  float *cs = nullptr, *sn = nullptr, *ctab = nullptr, *modtab = nullptr, *sbq = nullptr, *sbg = nullptr;
+  TRY(table(&cs, (size_t)S * (D / 2)));
+  TRY(table(&sn, (size_t)S * (D / 2)));
   launch_rope_table(cs, sn, S, D, P, k.rope_theta, st);
   if (kind == KIND_DENOISE) {
-    // c(t_k) of the Euler schedule: e(t_k) rows, z = swish(W_ti e + b), c = W_to z + b  (n <= 64 rows)
-    CK(cudaMalloc(&ctab, sizeof(float) * (size_t)n * w));
-    ge.owned.push_back(ctab);
+    // per Euler step t_k (n <= 64 rows): c(t_k) = W_to swish(W_ti e(t_k) + b_ti) + b_to; with Pi0's
+    // concat MLP instead the time half of its first layer, W_ti[:, w:] e(t_k) + b_ti; with the per-layer
+    // modulator also the modulation rows of every layer
+    TRY(table(&ctab, (size_t)n * w));
     launch_time_embedding(nullptr, n, n, ctx->e_tmp, w, st);
-    launch_linear<WT>(ctx->e_tmp, w, (const WT*)ctx->W.ti_w, ctx->W.ti_b, ctx->z_tmp, w, n, w, w, EPI_SWISH, st);
-    launch_linear<WT>(ctx->z_tmp, w, (const WT*)ctx->W.to_w, ctx->W.to_b, ctab, w, n, w, w, EPI_STORE, st);
+    if (tc == RTV_TIME_CONCAT) {
+      launch_rows_linear<WT>(ctx->e_tmp, w, (const WT*)ctx->W.ti_w + w, 2 * w, ctx->W.ti_b, 0, ctab, w, n, n, 0, n,
+                             w, w, EPI_STORE, st);
+    } else {
+      launch_linear<WT>(ctx->e_tmp, w, (const WT*)ctx->W.ti_w, ctx->W.ti_b, ctx->z_tmp, w, n, w, w, EPI_SWISH, st);
+      launch_linear<WT>(ctx->z_tmp, w, (const WT*)ctx->W.to_w, ctx->W.to_b, ctab, w, n, w, w, EPI_STORE, st);
+    }
+    if (tc == RTV_TIME_ADARMS) {
+      TRY(table(&modtab, (size_t)n * L * 6 * w));
+      if (ctx->use_fast) {
+        TRY(table(&sbq, (size_t)n * L * nq));
+        TRY(table(&sbg, (size_t)n * L * F2));
+      }
+      mod_tables<WT>(ctx, ctab, n, modtab, sbq, sbg, st);
+    }
   }
   CK(cudaGetLastError());
   CK(cudaStreamSynchronize(st));
@@ -171,20 +240,46 @@ rtv_status build_graph(rtv_ctx* ctx, int kind, int n, int batch, int P, GraphEnt
     if (fs == RTV_OK) fs = s2;
   };
   if (prologue) chain((*prologue)(st));
+  // what the embedding of a step adds to the action rows: c (RTV_TIME_ADD) or nothing
+  const bool add_c = tc == RTV_TIME_ADD;
   if (kind == KIND_DENOISE) {
     const float dt = (float)(1.0 / (double)n);
+    auto mod_of = [&](int step) {
+      ModTables m;
+      m.mod = modtab + (size_t)step * L * 6 * w;
+      m.sbq = sbq ? sbq + (size_t)step * L * nq : nullptr;
+      m.sbg = sbg ? sbg + (size_t)step * L * F2 : nullptr;
+      m.group_rows = 0;
+      return m;
+    };
     if (ctx->use_fast) {
       // step boundary k: head of step k-1 (k > 0) and embedding of step k (k < n)
-      chain(fast_step(ctx, batch, false, true, dt, ctab, 0, k.state_dim, false, st));
+      auto embed_tail = [&](int step) {
+        if (tc == RTV_TIME_CONCAT) {
+          concat_tokens<WT>(ctx, batch, ctab + (size_t)step * w, 0, st);
+          chain(fast_norm_rows(ctx, batch, st));
+        }
+      };
+      const float* g00 = tc == RTV_TIME_ADARMS ? modtab : nullptr;
+      chain(fast_step(ctx, batch, false, true, dt, add_c ? ctab : ctx->czero, 0, k.state_dim, false, st, g00, 0));
+      embed_tail(0);
       for (int step = 0; step < n && fs == RTV_OK; ++step) {
-        chain(fast_layers(ctx, batch, P, 1, cs, sn, st));
+        ModTables m;
+        if (tc == RTV_TIME_ADARMS) m = mod_of(step);
+        chain(fast_layers(ctx, batch, P, 1, cs, sn, st, tc == RTV_TIME_ADARMS ? &m : nullptr));
         const bool more = step + 1 < n;
-        chain(fast_step(ctx, batch, true, more, dt, more ? ctab + (size_t)(step + 1) * w : ctab, 0, k.state_dim,
-                        false, st));
+        const float* cnext = add_c ? (more ? ctab + (size_t)(step + 1) * w : ctab) : ctx->czero;
+        const float* g0 = (tc == RTV_TIME_ADARMS && more) ? modtab + (size_t)(step + 1) * L * 6 * w : nullptr;
+        chain(fast_step(ctx, batch, true, more, dt, cnext, 0, k.state_dim, false, st, g0, 0));
+        if (more) embed_tail(step + 1);
       }
     } else {
       for (int step = 0; step < n; ++step) {
-        simt_expert<WT>(ctx, batch, P, ctab + (size_t)step * w, 0, k.state_dim, 1, cs, sn, st);
+        ModTables m;
+        if (tc == RTV_TIME_ADARMS) m = mod_of(step);
+        simt_expert<WT>(ctx, batch, P, add_c ? ctab + (size_t)step * w : ctx->czero, 0, k.state_dim, 1, cs, sn, st,
+                        tc == RTV_TIME_CONCAT ? ctab + (size_t)step * w : nullptr, 0,
+                        tc == RTV_TIME_ADARMS ? &m : nullptr);
         launch_out_head<WT>(ctx->h, ctx->W.g_final, (const WT*)ctx->W.ao_w, ctx->W.ao_b, ctx->x, nullptr, dt, batch,
                             w, S, k.action_dim, k.rms_eps, ctx->status, st);
       }
@@ -192,13 +287,37 @@ rtv_status build_graph(rtv_ctx* ctx, int kind, int n, int batch, int P, GraphEnt
   } else {
     const int T = n;
     launch_verify_interp(ctx->draft, ctx->eps, ctx->taus, ctx->x, T, ctx->H * k.action_dim, st);
-    time_condition<WT>(ctx, ctx->taus, T, 0, ctx->c_verify, st);
+    // one flow time per suffix group: c(tau_i) rows (or the concat MLP's time half), and the
+    // modulation rows of every layer
+    if (tc == RTV_TIME_CONCAT) {
+      launch_time_embedding(ctx->taus, T, 0, ctx->e_tmp, w, st);
+      launch_rows_linear<WT>(ctx->e_tmp, w, (const WT*)ctx->W.ti_w + w, 2 * w, ctx->W.ti_b, 0, ctx->c_verify, w, T,
+                             T, 0, T, w, w, EPI_STORE, st);
+    } else {
+      time_condition<WT>(ctx, ctx->taus, T, 0, ctx->c_verify, st);
+    }
+    ModTables m;
+    if (tc == RTV_TIME_ADARMS) {
+      mod_tables<WT>(ctx, ctx->c_verify, T, ctx->mod_v, ctx->use_fast ? ctx->sbq_v : nullptr,
+                     ctx->use_fast ? ctx->sbg_v : nullptr, st);
+      m.mod = ctx->mod_v;
+      m.sbq = ctx->sbq_v;
+      m.sbg = ctx->sbg_v;
+      m.group_rows = 1;
+    }
+    const ModTables* mp = tc == RTV_TIME_ADARMS ? &m : nullptr;
     if (ctx->use_fast) {
-      chain(fast_step(ctx, T, false, true, 0.f, ctx->c_verify, w, 0, false, st));
-      chain(fast_layers(ctx, T, P, 0, cs, sn, st));
+      chain(fast_step(ctx, T, false, true, 0.f, add_c ? ctx->c_verify : ctx->czero, add_c ? w : 0, 0, false, st,
+                      mp ? ctx->mod_v : nullptr, mp ? L * 6 * w : 0));
+      if (tc == RTV_TIME_CONCAT) {
+        concat_tokens<WT>(ctx, T, ctx->c_verify, w, st);
+        chain(fast_norm_rows(ctx, T, st));
+      }
+      chain(fast_layers(ctx, T, P, 0, cs, sn, st, mp));
       chain(fast_step(ctx, T, true, false, 0.f, ctx->c_verify, w, 0, true, st));
     } else {
-      simt_expert<WT>(ctx, T, P, ctx->c_verify, w, 0, 0, cs, sn, st);
+      simt_expert<WT>(ctx, T, P, add_c ? ctx->c_verify : ctx->czero, add_c ? w : 0, 0, 0, cs, sn, st,
+                      tc == RTV_TIME_CONCAT ? ctx->c_verify : nullptr, w, mp);
       launch_out_head<WT>(ctx->h, ctx->W.g_final, (const WT*)ctx->W.ao_w, ctx->W.ao_b, ctx->x, ctx->v, 0.f, T, w,
                           S, k.action_dim, k.rms_eps, ctx->status, st);
     }
@@ -305,6 +424,13 @@ rtv_status ctx_create(const rtv_expert_config& k, int cuda_device, int S, bool b
   A(&ctx->taus, (size_t)(ctx->Gmax > 0 ? ctx->Gmax : 1));
   A(&ctx->vparams, 4);
   A(&ctx->dist, (size_t)(ctx->Gmax > 0 ? ctx->Gmax : 1) * H);
+  A(&ctx->czero, (size_t)w);
+  if (k.time_cond == RTV_TIME_ADARMS) {
+    const size_t G1 = ctx->Gmax > 0 ? ctx->Gmax : 1, L = k.n_layers;
+    A(&ctx->mod_v, G1 * L * 6 * w);
+    A(&ctx->sbq_v, G1 * L * (ctx->Q + 2 * ctx->KV));
+    A(&ctx->sbg_v, G1 * L * 2 * F);
+  }
   if (s == RTV_OK) s = dev_alloc_t(ctx, &ctx->accepted, 1);
   if (s == RTV_OK) s = dev_alloc_t(ctx, &ctx->flags, 1);
   if (s == RTV_OK) s = dev_alloc_t(ctx, &ctx->status, 1);
@@ -313,6 +439,7 @@ rtv_status ctx_create(const rtv_expert_config& k, int cuda_device, int S, bool b
     s = dev_alloc(ctx, &kvp, (size_t)k.n_layers * 2 * k.max_batch * k.n_kv_heads * k.max_prefix_len * D * ctx->elt);
   ctx->prefix_kv = kvp;
   if (s == RTV_OK && cudaMemset(ctx->status, 0, sizeof(unsigned)) != cudaSuccess) s = RTV_ERR_CUDA;
+  if (s == RTV_OK && cudaMemset(ctx->czero, 0, sizeof(float) * w) != cudaSuccess) s = RTV_ERR_CUDA;
   if (s == RTV_OK && cudaStreamCreateWithFlags(&ctx->cap_stream, cudaStreamNonBlocking) != cudaSuccess)
     s = RTV_ERR_CUDA;
   if (s == RTV_OK && k.dtype == RTV_BF16) {
@@ -334,8 +461,14 @@ void add_layer_slots(rtv_ctx* ctx, SlotTable& slots, const std::string& p, Layer
   const long long w = k.width, F = k.mlp_dim, Q = ctx->Q, KV = ctx->KV;
   const int md = k.dtype;
   const size_t e = ctx->elt;
-  slots[p + "attn_norm.g"] = ParamSlot{{w}, RTV_F32, (void**)&L.g_attn, 0, nullptr, 0};
-  slots[p + "mlp_norm.g"] = ParamSlot{{w}, RTV_F32, (void**)&L.g_mlp, 0, nullptr, 0};
+  if (k.time_cond == RTV_TIME_ADARMS) {
+    // the per-layer time modulator replaces the two norm gains
+    slots[p + "time_mod.w"] = ParamSlot{{6 * w, w}, md, &L.tmod_w, 0, nullptr, 0};
+    slots[p + "time_mod.b"] = ParamSlot{{6 * w}, RTV_F32, (void**)&L.tmod_b, 0, nullptr, 0};
+  } else {
+    slots[p + "attn_norm.g"] = ParamSlot{{w}, RTV_F32, (void**)&L.g_attn, 0, nullptr, 0};
+    slots[p + "mlp_norm.g"] = ParamSlot{{w}, RTV_F32, (void**)&L.g_mlp, 0, nullptr, 0};
+  }
   const size_t qkv_bytes = (size_t)(Q + 2 * KV) * w * e;
   slots[p + "q_proj.w"] = ParamSlot{{Q, w}, md, nullptr, 0, &L.qkv, qkv_bytes};
   slots[p + "k_proj.w"] = ParamSlot{{KV, w}, md, nullptr, (size_t)Q * w * e, &L.qkv, qkv_bytes};
@@ -417,6 +550,10 @@ rtv_status rtv_create(const rtv_expert_config* cfg_in, int cuda_device, rtv_ctx*
   // FP8 E4M3 MLP weights ride on bf16 activations (tensor-core path only)
   if (k.mlp_dtype != k.dtype && !(k.mlp_dtype == RTV_FP8_E4M3 && k.dtype == RTV_BF16)) return RTV_ERR_UNSUPPORTED;
   if (k.suffix_mask != RTV_MASK_BIDIR && k.suffix_mask != RTV_MASK_PI0_BLOCK) return RTV_ERR_ARG;
+  if (k.time_cond != RTV_TIME_ADD && k.time_cond != RTV_TIME_CONCAT && k.time_cond != RTV_TIME_ADARMS)
+    return RTV_ERR_ARG;
+  // the modulator's shift terms are taken from the bf16/fp32 gate/up rows
+  if (k.time_cond == RTV_TIME_ADARMS && k.mlp_dtype == RTV_FP8_E4M3) return RTV_ERR_UNSUPPORTED;
   if (!(k.rms_eps >= 0.f) || !(k.rope_theta >= 0.f)) return RTV_ERR_ARG;
   if (k.barrier_timeout_ns <= 0) k.barrier_timeout_ns = 100000000LL;
 
@@ -451,7 +588,7 @@ rtv_status rtv_load_expert(rtv_ctx* ctx, const rtv_tensor* params, int n_params)
   vec("state_proj.b", w, &W.sp_b);
   mat("action_in_proj.w", w, A, &W.ai_w);
   vec("action_in_proj.b", w, &W.ai_b);
-  mat("time_mlp_in.w", w, w, &W.ti_w);
+  mat("time_mlp_in.w", w, k.time_cond == RTV_TIME_CONCAT ? 2 * w : w, &W.ti_w);
   vec("time_mlp_in.b", w, &W.ti_b);
   mat("time_mlp_out.w", w, w, &W.to_w);
   vec("time_mlp_out.b", w, &W.to_b);

@@ -24,6 +24,8 @@ struct LayerW {
   float* down_s = nullptr;   // [w] per-row scales of down (FP8 MLP only)
   float* g_attn = nullptr;
   float* g_mlp = nullptr;
+  void* tmod_w = nullptr;  // [6w][w] per-layer time modulator (RTV_TIME_ADARMS)
+  float* tmod_b = nullptr; // [6w]
 };
 
 struct ExpertW {
@@ -59,6 +61,19 @@ struct ParamSlot {
 };
 using SlotTable = std::unordered_map<std::string, ParamSlot>;
 
+// Per-layer time modulation tables (RTV_TIME_ADARMS), rows of all layers:
+// mod [.][L][6w] = (scale_a, shift_a, gate_a, scale_m, shift_m, gate_m) of
+// every layer, sbq [.][L][Q+2KV] = W_qkv . shift_a and sbg [.][L][2F] =
+// W_gu . shift_m (natural row order; the shifts' share of the projections).
+// group_rows 0: every suffix group reads row 0 (one flow time for the
+// batch); 1: group g reads row g (one flow time per verification tau).
+struct ModTables {
+  const float* mod = nullptr;
+  const float* sbq = nullptr;
+  const float* sbg = nullptr;
+  int group_rows = 0;
+};
+
 // Work captured at the head of a graph, before the denoising loop.
 using GraphPrologue = std::function<rtv_status(cudaStream_t)>;
 
@@ -89,6 +104,9 @@ struct rtv_ctx {
   float *x = nullptr, *v = nullptr, *state = nullptr;
   float *e_tmp = nullptr, *z_tmp = nullptr, *c_verify = nullptr;
   float *draft = nullptr, *eps = nullptr, *taus = nullptr, *vparams = nullptr, *dist = nullptr;
+  float* czero = nullptr;   // [w] zeros: the time condition of the variants that add none to the tokens
+  // RTV_TIME_ADARMS verification tables (one row per tau): see ModTables
+  float *mod_v = nullptr, *sbq_v = nullptr, *sbg_v = nullptr;
   int* accepted = nullptr;
   unsigned* flags = nullptr;
   unsigned* status = nullptr;
@@ -116,6 +134,6 @@ rtv_status capture_denoise(rtv_ctx* ctx, int n_steps, int P, const GraphPrologue
 // The SIMT layers over G suffixes of ctx->S rows (residual stream ctx->h).
 template <typename WT>
 void simt_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, const float* rope_cs, const float* rope_sn,
-                 cudaStream_t st);
+                 cudaStream_t st, const ModTables* mod = nullptr);
 
 }  // namespace rtv

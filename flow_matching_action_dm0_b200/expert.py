@@ -22,6 +22,7 @@ from . import _lib as L
 
 _DTYPES = {"f32": L.RTV_F32, "bf16": L.RTV_BF16, "fp8_e4m3": L.RTV_FP8_E4M3, "same": L.RTV_SAME}
 _MASKS = {"bidir": L.RTV_MASK_BIDIR, "pi0_block": L.RTV_MASK_PI0_BLOCK}
+_TIME = {"add": L.RTV_TIME_ADD, "concat": L.RTV_TIME_CONCAT, "adarms": L.RTV_TIME_ADARMS}
 
 
 def make_config(shape, max_batch: Optional[int] = None, max_taus: int = 4,
@@ -40,6 +41,7 @@ def make_config(shape, max_batch: Optional[int] = None, max_taus: int = 4,
     cfg.rms_eps = float(g("rms_eps", 1e-6))
     cfg.rope_theta = float(g("rope_theta", 10000.0))
     cfg.barrier_timeout_ns = 0
+    cfg.time_cond = _TIME[g("time_cond", "add")]
     return cfg
 
 

@@ -65,6 +65,14 @@ typedef enum {
   RTV_MASK_PI0_BLOCK = 1   /* the state token does not see the action tokens          */
 } rtv_suffix_mask;
 
+/* How the flow time t enters the expert ([DM0.5] 5.2 names time_mlp_in/out
+ * and a per-layer time modulator; the forms are readings of the pages). */
+typedef enum {
+  RTV_TIME_ADD = 0,      /* c(t) = W_to swish(W_ti e(t) + b_ti) + b_to added to every action token     */
+  RTV_TIME_CONCAT = 1,   /* Pi0: action token = W_to swish(W_ti [W_ai x + b_ai ; e(t)] + b_ti) + b_to  */
+  RTV_TIME_ADARMS = 2    /* DM0.5: per layer, (scale, shift, gate) of each norm's branch from c(t)     */
+} rtv_time_cond;
+
 /* Device status bits (rtv_device_status). */
 #define RTV_DEV_TIMEOUT  0x1u   /* a bounded spin-wait in a kernel gave up   */
 #define RTV_DEV_NUMERIC  0x2u   /* a NaN/Inf reached the action output       */
@@ -91,7 +99,12 @@ typedef enum {
  * widened to bf16 exactly).  A shape the tensor-core path does not take
  * returns RTV_ERR_UNSUPPORTED from rtv_create for an FP8 MLP.
  * rope_theta 0 disables rotary embedding.  barrier_timeout_ns bounds every
- * device-side wait (0 = library default, 100 ms).
+ * device-side wait (0 = library default, 100 ms).  time_cond selects how the
+ * flow time conditions the expert (rtv_time_cond); with RTV_TIME_ADARMS,
+ * layer l's norms become x / rms(x) * (1 + scale) + shift for every suffix
+ * token and its two branches are multiplied by their gates, where
+ * (scale_a, shift_a, gate_a, scale_m, shift_m, gate_m) =
+ * layers.l.time_mod.w . c(t) + layers.l.time_mod.b, in that order.
  */
 typedef struct {
   int n_layers, width, n_q_heads, n_kv_heads, head_dim, mlp_dim;
@@ -103,6 +116,7 @@ typedef struct {
   float rms_eps;
   float rope_theta;
   long long barrier_timeout_ns;
+  int time_cond;       /* rtv_time_cond (RTV_TIME_ADD = 0 by default)                       */
 } rtv_expert_config;
 
 /*
@@ -120,6 +134,10 @@ typedef struct {
  *   layers.l.gate_proj.s [F]  layers.l.up_proj.s [F]  layers.l.down_proj.s [w]
  *        (fp32 per-row scales, only with mlp_dtype = RTV_FP8_E4M3)
  *   final_norm.g [w]  action_out_proj.w [A][w]  action_out_proj.b [A]
+ * With time_cond RTV_TIME_CONCAT, time_mlp_in.w is [w][2w] (its first w
+ * columns read the action embedding, the last w the sinusoid e(t)).  With
+ * RTV_TIME_ADARMS, every layer has layers.l.time_mod.w [6w][w] and
+ * layers.l.time_mod.b [6w] instead of layers.l.attn_norm.g and mlp_norm.g.
  * Matrices must be given in the config dtype (or RTV_FP8_E4M3 for the MLP
  * when mlp_dtype says so); vectors in RTV_F32.
  */

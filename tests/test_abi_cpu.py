@@ -50,6 +50,17 @@ def test_invalid_config_is_refused_before_device_use():
     assert not h.value
 
 
+@pytest.mark.parametrize("value", [3, -1])
+def test_invalid_time_condition_is_refused_before_device_use(value):
+    from synthetic import get_config
+    from flow_matching_action_dm0_b200 import make_config
+    cfg = make_config(get_config("tiny-fp32"))
+    cfg.time_cond = value
+    h = C.c_void_p()
+    assert L.load_library().rtv_create(C.byref(cfg), 0, C.byref(h)) == L.RTV_ERR_ARG
+    assert not h.value
+
+
 def test_create_without_gpu_reports_cuda_error():
     import torch
     if torch.cuda.is_available():
