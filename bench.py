@@ -74,13 +74,18 @@ def parse_args(argv=None):
 def algorithmic_bytes_per_step(cfg, batch=1):
     """Weight bytes of every layer and of the state/action projections, plus
     the prefix K and V of every layer, each counted once per Euler step.
-    The time MLP depends only on t and is precomputed, so it is excluded."""
+    The time MLP depends only on t and is precomputed, so it is excluded, and
+    so are the per-layer time modulator's weights (its rows and shift terms
+    are tables of the Euler schedule); Pi0's concat time MLP reads its
+    action half (w x w) and output layer (w x w) every step."""
     elt = 4 if cfg.dtype == "f32" else 2
     w, f = cfg.width, cfg.mlp_dim
     mlp_elt = 1 if cfg.mlp_dtype == "fp8_e4m3" else elt
     attn = w * (cfg.q_dim + 2 * cfg.kv_dim) + cfg.q_dim * w
     layer = attn * elt + 3 * w * f * mlp_elt
     proj = (w * cfg.state_dim + w * cfg.action_dim + cfg.action_dim * w) * elt
+    if getattr(cfg, "time_cond", "add") == "concat":
+        proj += 2 * w * w * elt
     kv = 2 * batch * cfg.prefix_len * cfg.kv_dim * elt
     return cfg.n_layers * (layer + kv) + proj
 
@@ -218,14 +223,57 @@ def run_reference_draft(args, info):
     print(json.dumps(line), flush=True)
 
 
+def run_reference_prefill(args, info):
+    """The CPU oracle on the gemma2b-prefill workload, bounded: each step is a
+    2-layer oracle prefill over the 816 tokens (one full layer and the last
+    layer's K/V, weight generation included) scaled to the stack's depth,
+    plus one oracle Euler step of the pi0-bf16 expert scaled to the chunk."""
+    from oracle import expert as O
+    from oracle import prefill as OP
+    from synthetic import (get_config, get_prefill_config, make_noise, make_prefill_weights, make_prefix_embeddings,
+                           make_prefix_kv, make_state, make_weights)
+    pc = get_prefill_config(args.workload)
+    cfg = get_config("pi0-bf16", n_steps=args.n_steps, prefix_len=pc.n_tokens)
+    two = pc.with_(n_layers=2)
+    emb = make_prefix_embeddings(pc)
+    W = O.to_f64(make_weights(cfg))
+    kv = make_prefix_kv(cfg)
+    pk, pv = kv[:, 0, 0].astype(np.float64), kv[:, 1, 0].astype(np.float64)
+    x = make_noise(cfg)[0].astype(np.float64)
+    state = make_state(cfg)[0]
+    steps = max(1, min(args.steps, 2))
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        OP.prefill_kv(lambda l: make_prefill_weights(two, layers=[l]), two, emb)
+    t_pre = (time.perf_counter() - t0) / steps
+    t0 = time.perf_counter()
+    O.expert_velocity(W, cfg, x, state, 1.0, pk, pv)
+    t_step = time.perf_counter() - t0
+    us = (t_pre * (pc.n_layers - 1) + t_step * cfg.n_steps) * 1e6
+    line = {
+        "impl": "reference", "metric": PREFILL_METRIC, "value": us, "unit": "us", "n_gpus": args.gpus,
+        "steps": steps, "warmup": 0, "ms_per_step": us / 1000.0, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "n_tokens": pc.n_tokens, "expert": "pi0-bf16", "n_steps": cfg.n_steps},
+        "cpu_baseline": {"value": us, "unit": "us", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"{steps} 2-layer oracle prefills scaled to {pc.n_layers} layers + one oracle "
+                                   f"Euler step scaled x{cfg.n_steps}"},
+        "e2e": {"value": us, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(args, info):
     """The CPU oracle, as it stands, on a bounded sample of the workload:
     each step is one Euler step of the chunk, scaled to chunk latency."""
     if not info.is_main:
         return
-    from synthetic import DRAFTS
+    from synthetic import DRAFTS, PREFILLS
     if args.workload in DRAFTS:
         run_reference_draft(args, info)
+        return
+    if args.workload in PREFILLS:
+        run_reference_prefill(args, info)
         return
     from synthetic import get_config
     cfg = get_config(args.workload, n_steps=args.n_steps)

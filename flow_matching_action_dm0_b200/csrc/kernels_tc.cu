@@ -113,7 +113,7 @@ struct GemmArgs {
   unsigned long long* trace;  // optional phase stamps [cta][16] (globaltimer ns), or nullptr
   long long timeout_ns;
   int T, n_mma, kslice, stages, w, S, Hq, Hkv, D, F, K, w_tile0;
-  int tt;                     // token rows per CTA (a multiple of 16, <= 256); blockIdx.z picks the tile
+  int tt;                     // token rows per CTA (a multiple of 16, <= 256); blockIdx.y picks the tile
   int nt_base;                // first 128-row weight tile of the grid within the layer (QKV: K/V tiles only)
   int kv_rows;                // row stride of ks / vs per (sequence, kv head)
   int seq;                    // QKV: tokens of one sequence -- RoPE position and ks/vs row are t % seq, the
@@ -214,11 +214,13 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
   extern __shared__ uint8_t smem_raw[];
   constexpr int kMaxOwn = 160;   // tokens one rank reduces and finishes
   __shared__ float rs_s[kMaxOwn];
-  // Token tiling: blockIdx.z takes token rows [t0, t0 + n_mma) of the tiled
-  // activation layout, which has n_rows rows per 64-column block; T of them are
-  // real tokens.
+  // Grid (K slice, token tile, weight tile): blockIdx.y takes token rows
+  // [t0, t0 + n_mma) of the tiled activation layout, which has n_rows rows
+  // per 64-column block (T of them real tokens); the token tiles of one
+  // weight tile are adjacent in launch order, so they share its weight
+  // boxes through L2.
   const int n_rows = a.n_mma;
-  const int t0 = (int)blockIdx.z * a.tt;
+  const int t0 = (int)blockIdx.y * a.tt;
   const int n_mma = min(a.tt, n_rows - t0);
   const int T = min(a.T - t0, n_mma);
   const int cs = gridDim.x;
@@ -233,7 +235,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = ptx::cluster_ctarank();
-  const int nt = (int)blockIdx.y + a.nt_base;
+  const int nt = (int)blockIdx.z + a.nt_base;
   const int nbox = a.kslice >> 6;
   const int NS = L.stages;
   const int k0 = (int)rank * a.kslice;
@@ -287,11 +289,12 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
         else ptx::bulk_load_hint(base + b * L.stage_bytes, wsrc + (size_t)b * 8192, 16384u, &full[b], pol);
       }
       if (trace) trace[TR_W_ISSUED] = ptx::globaltimer();
-    } else if (lane == 2 && a.pf) {
-      // this CTA's share of the next projection's weights, into L2 (a hint)
-      const unsigned long long n_cta = (unsigned long long)gridDim.x * gridDim.y;
+    } else if (lane == 2 && a.pf && blockIdx.y == 0) {
+      // this CTA's share of the next projection's weights, into L2 (a hint;
+      // the CTAs of the first token tile split it)
+      const unsigned long long n_cta = (unsigned long long)gridDim.x * gridDim.z;
       const unsigned long long share = ((a.pf_bytes + n_cta - 1) / n_cta + 15) & ~15ull;
-      const unsigned long long lo = share * ((unsigned long long)blockIdx.y * gridDim.x + blockIdx.x);
+      const unsigned long long lo = share * ((unsigned long long)blockIdx.z * gridDim.x + blockIdx.x);
       const unsigned long long hi = lo + share < a.pf_bytes ? lo + share : a.pf_bytes;
       for (unsigned long long off = lo; off < hi; off += 32768)
         ptx::prefetch_l2_bulk(a.pf + off, (uint32_t)(hi - off < 32768 ? hi - off : 32768));
@@ -483,7 +486,6 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
 #pragma unroll 1
     for (int tl = ew; tl < n_own; tl += kEpiWarps) {
       const int t = t0 + t_own0 + tl;   // global token row
-      const int tg = t / a.S;           // its suffix group
       float2 x1 = make_float2(0.f, 0.f), x2 = make_float2(0.f, 0.f);
       for (int qr = 0; qr < cs; ++qr) {
         const float* rr = recv + (qr * per + tl) * 128;
@@ -501,7 +503,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
         x2.y *= ws2.y;
       }
       if ((MODE == GM_O || MODE == GM_DOWN) && a.gate) {   // gated branch (time modulator)
-        const float* gp = a.gate + (size_t)tg * a.gate_stride;
+        const float* gp = a.gate + (size_t)(t / a.S) * a.gate_stride;
         const float2 q1 = *reinterpret_cast<const float2*>(gp + n1);
         const float2 q2 = *reinterpret_cast<const float2*>(gp + n2);
         x1.x *= q1.x;
@@ -510,8 +512,9 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
         x2.y *= q2.y;
       }
       if ((MODE == GM_O || MODE == GM_DOWN) && a.g_next && a.g_stride) {   // per-group gain of the next norm
-        gn1 = *reinterpret_cast<const float2*>(a.g_next + (size_t)tg * a.g_stride + n1);
-        gn2 = *reinterpret_cast<const float2*>(a.g_next + (size_t)tg * a.g_stride + n2);
+        const float* gg = a.g_next + (size_t)(t / a.S) * a.g_stride;
+        gn1 = *reinterpret_cast<const float2*>(gg + n1);
+        gn2 = *reinterpret_cast<const float2*>(gg + n2);
       }
       if (MODE == GM_O || MODE == GM_DOWN) {
         // residual add, then the next norm's bf16 input and this tile's sum of squares
@@ -540,20 +543,19 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
         x2.x *= rs;
         x2.y *= rs;
         if (a.sb) {   // the modulator's shift carried through the projection (natural row order)
-          const float* sp = a.sb + (size_t)tg * a.sb_stride;
+          const float* sbp = a.sb + (size_t)(t / a.S) * a.sb_stride;
           const int r1 = MODE == GM_GU ? 64 * nt + f0 : hh * a.D + dq0 + f0;
           const int r2 = MODE == GM_GU ? a.F + 64 * nt + f0 : hh * a.D + dq0 + hd + f0;
-          x1.x += sp[r1];
-          x1.y += sp[r1 + 1];
-          x2.x += sp[r2];
-          x2.y += sp[r2 + 1];
+          x1.x += sbp[r1];
+          x1.y += sbp[r1 + 1];
+          x2.x += sbp[r2];
+          x2.y += sbp[r2 + 1];
         }
         if (MODE == GM_GU) {
           *reinterpret_cast<uint32_t*>(a.m + ts_offset(t, nt * 64 + f0, n_rows)) =
               ptx::pack_bf16x2(gelu_tanh(x1.x) * x2.x, gelu_tanh(x1.y) * x2.y);
         } else {
           const int g = t / a.S, s = t - g * a.S;           // suffix group and row (q and suffix K/V tiles)
-          const int sq = t / a.seq, sp = t - sq * a.seq;    // sequence and position (K/V rows)
           float2 y1 = x1, y2 = x2;
           if (rope) {
             const float2 c = *reinterpret_cast<const float2*>(in_s + tl * 128 + f0);
@@ -580,6 +582,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
               dst[ts_offset(d2 + 1, s, a.D)] = __float2bfloat16_rn(y2.y);
             }
           } else {
+            const int sq = t / a.seq, sp = t - sq * a.seq;    // sequence and position (K/V rows)
             __nv_bfloat16* dst;
             if (hh < a.Hq) dst = a.q + ((size_t)t * a.Hq + hh) * a.D;
             else if (hh < a.Hq + a.Hkv) dst = a.ks + (((size_t)sq * a.Hkv + (hh - a.Hq)) * a.kv_rows + sp) * a.D;
@@ -1565,7 +1568,7 @@ cudaError_t launch_gemm(const GemmArgs& a, const GemmPlan& pl, cudaStream_t st,
                         unsigned long long pf_cap = ~0ull) {
   auto kern = gemm_tc_kernel<MODE>;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(pl.cs, pl.n_tiles, pl.n_tt);
+  cfg.gridDim = dim3(pl.cs, pl.n_tt, pl.n_tiles);
   cfg.blockDim = dim3(kGemmThreads, 1, 1);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = st;
