@@ -44,7 +44,7 @@ def _draft(dcfg, weights=None, batch=1, n_vis=None, max_vis=None):
     return got, ref, path
 
 
-@pytest.mark.parametrize("batch,n_vis", [(1, 64), (2, 37)])
+@pytest.mark.parametrize("batch,n_vis", [(1, 64), (2, 37), (1, 1)])
 def test_fp32_draft_matches_oracle(cuda_ok, batch, n_vis):
     dcfg = get_draft_config("draft-tiny")
     got, ref, path = _draft(dcfg, batch=batch, n_vis=n_vis)
@@ -58,7 +58,7 @@ def test_fp32_draft_without_rope_and_two_kv_heads(cuda_ok):
     assert np.max(np.abs(got - ref)) <= 1e-4
 
 
-@pytest.mark.parametrize("batch,n_vis", [(1, 100), (2, 64), (3, 130)])
+@pytest.mark.parametrize("batch,n_vis", [(1, 100), (2, 64), (3, 130), (1, 1)])
 def test_bf16_draft_tensor_cores_match_oracle(cuda_ok, batch, n_vis):
     dcfg = get_draft_config("flash-draft", **SMALL_BF16)
     got, ref, path = _draft(dcfg, batch=batch, n_vis=n_vis)

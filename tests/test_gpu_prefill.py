@@ -58,10 +58,10 @@ def _expert_and_stack(n_layers, width, n_q_heads, mlp_dim, n_tokens):
     return cfg, pc
 
 
-@pytest.mark.parametrize("n_tokens", [150, 64, 37])
+@pytest.mark.parametrize("n_tokens", [150, 64, 37, 1])
 def test_prefill_denoise_matches_oracle_small(cuda_ok, n_tokens):
     """Two layers, width 512: ragged query groups (150 = 2 x 64 + 22), one
-    exact group, one partial group."""
+    exact group, one partial group, a single token."""
     cfg, pc = _expert_and_stack(2, 512, 2, 2048, n_tokens)
     ex, pf, We, emb, noise, state, got = _run(cfg, pc, 3)
     ref = OP.prefill_denoise(provider(pc), pc, We, cfg, emb, noise, state, 3)[0]
