@@ -35,10 +35,13 @@ Readings where the pages are silent (the plainest one in each case):
       reuses the cached prefix (the observation's VLM prefill is outside the
       suffix loop).  On acceptance the returned chunk is the draft; the
       accepted length says how much of it the caller may execute.
-Pins (tests/test_oracle_pins.py): the zero-block closed form (all block
-matrices zero -> head applied to the queries), invariance to the order of
-the visual tokens without RoPE, equivariance in the query order without
-RoPE, an independent PyTorch statement, and both branches of the round.
+Pins (tests/test_oracle_draft_pins.py): the zero-block closed form (all
+block matrices zero -> head applied to the queries), invariance to the order
+of the visual tokens without RoPE, equivariance in the query order without
+RoPE, an independent PyTorch statement, and every branch of the round.
+draft_forward with random weights: parity unpinned by the pages (they print
+no worked example); pinned only through those closed forms, symmetries and
+the independent statement.
 """
 
 from __future__ import annotations

@@ -24,10 +24,11 @@ Readings where the pages are silent (the plainest one in each case):
       as many layers as the expert and the same kv heads and head_dim.  The
       last layer's attention output and MLP feed nothing and are not
       computed.
-Pins (tests/test_oracle_prefill_pins.py): the one-layer closed form, token
-permutation equivariance without RoPE, the single-token closed form, an
-independent PyTorch statement, and prefill + denoise = denoise on the
-prefill's cache.
+Pins (tests/test_oracle_prefill_pins.py): the zero-first-layer closed form,
+token permutation equivariance without RoPE, the single-token closed form,
+an independent PyTorch statement, and prefill + denoise = denoise on the
+prefill's cache.  prefill_kv with random weights: parity unpinned by the
+pages (no worked example); pinned only through those.
 """
 
 from __future__ import annotations
