@@ -74,19 +74,6 @@ rtv_status dfail(rtv_draft* d, rtv_status s, const std::string& msg) {
     if (_s != RTV_OK) return _s;       \
   } while (0)
 
-struct DevGuard {
-  int prev = -1;
-  explicit DevGuard(int dev) {
-    cudaGetDevice(&prev);
-    if (prev != dev) cudaSetDevice(dev);
-  }
-  ~DevGuard() {
-    int cur = -1;
-    cudaGetDevice(&cur);
-    if (prev >= 0 && cur != prev) cudaSetDevice(prev);
-  }
-};
-
 rtv_status dalloc(rtv_draft* d, void** p, size_t bytes, bool zero = false) {
   *p = nullptr;
   if (bytes == 0) bytes = 16;
@@ -180,19 +167,6 @@ __global__ void vis_kv_store_kernel(const float* __restrict__ kv, const float* _
   }
 }
 
-int count_kernels(cudaGraph_t g) {
-  size_t n = 0;
-  if (cudaGraphGetNodes(g, nullptr, &n) != cudaSuccess) return -1;
-  std::vector<cudaGraphNode_t> nodes(n);
-  cudaGraphGetNodes(g, nodes.data(), &n);
-  int k = 0;
-  for (auto nd : nodes) {
-    cudaGraphNodeType t;
-    if (cudaGraphNodeGetType(nd, &t) == cudaSuccess && t == cudaGraphNodeTypeKernel) ++k;
-  }
-  return k;
-}
-
 // The draft forward for (V, B), enqueued on st (captured into a graph).
 template <typename WT>
 rtv_status enqueue_forward(rtv_draft* d, int V, int B, const float* cs_v, const float* sn_v, const float* cs_q,
@@ -264,7 +238,7 @@ rtv_status build_graph(rtv_draft* d, int V, int B, GraphEntry& ge) {
                                       cudaGetErrorString(e1 != cudaSuccess ? e1 : e2));
   }
   ge.graph = g;
-  ge.kernels = count_kernels(g);
+  ge.kernels = count_kernel_nodes(g);
   DCK(cudaGraphInstantiate(&ge.exec, g, 0));
   DCK(cudaGraphUpload(ge.exec, st));
   DCK(cudaStreamSynchronize(st));
@@ -346,7 +320,7 @@ rtv_status rtv_draft_create(const rtv_draft_config* cfg, int cuda_device, rtv_dr
   d->cfg = c;
   d->device = cuda_device;
   d->elt = c.dtype == RTV_F32 ? 4 : 2;
-  DevGuard dg(cuda_device);
+  DeviceGuard dg(cuda_device);
   rtv_status s = ctx_create(k, cuda_device, c.n_queries, true, &d->blk);
   const size_t w = c.width, Tv = (size_t)c.max_batch * c.max_vis, KV = (size_t)c.n_kv_heads * c.head_dim;
   auto A = [&](void** p, size_t bytes, bool zero = false) {
@@ -375,7 +349,7 @@ rtv_status rtv_draft_load(rtv_draft* d, const rtv_tensor* params, int n_params) 
   if (!d) return RTV_ERR_ARG;
   if (!params || n_params <= 0) return dfail(d, RTV_ERR_ARG, "no parameters");
   if (d->loaded) return dfail(d, RTV_ERR_STATE, "draft model already loaded");
-  DevGuard dg(d->device);
+  DeviceGuard dg(d->device);
   rtv_ctx* c = d->blk;
   const long long w = d->cfg.width, H = d->cfg.n_queries, A = d->cfg.action_dim;
   c->W.layers.assign(1, LayerW());
@@ -406,7 +380,7 @@ rtv_status rtv_draft_forward(rtv_draft* d, const void* vis, int n_vis, int batch
                              rtv_stream stream) {
   if (!d) return RTV_ERR_ARG;
   if (!chunk_out) return dfail(d, RTV_ERR_ARG, "null output");
-  DevGuard dg(d->device);
+  DeviceGuard dg(d->device);
   cudaStream_t st = (cudaStream_t)stream;
   DTRY(forward_to_out(d, vis, n_vis, batch, st));
   DCK(cudaMemcpyAsync(chunk_out, d->out, (size_t)batch * d->cfg.n_queries * d->cfg.action_dim * sizeof(float),
@@ -426,7 +400,7 @@ rtv_status rtv_flash_round(rtv_ctx* ctx, rtv_draft* d, const void* vis, int n_vi
     return dfail(d, RTV_ERR_SHAPE, "the draft chunk shape differs from the expert's");
   if (ctx->have_prefix && ctx->prefix_batch != 1)
     return dfail(d, RTV_ERR_SHAPE, "a round serves one observation: install a prefix of batch 1");
-  DevGuard dg(d->device);
+  DeviceGuard dg(d->device);
   cudaStream_t st = (cudaStream_t)stream;
   // fast path: draft, then verification of the chunk left in d->out
   DTRY(forward_to_out(d, vis, n_vis, 1, st));
@@ -471,7 +445,7 @@ int rtv_draft_kernel_count(rtv_draft* d, int n_vis, int batch) {
 
 void rtv_draft_destroy(rtv_draft* d) {
   if (!d) return;
-  DevGuard dg(d->device);
+  DeviceGuard dg(d->device);
   cudaDeviceSynchronize();
   for (auto& kv : d->graphs) {
     if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);

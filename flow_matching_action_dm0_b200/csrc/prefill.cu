@@ -64,32 +64,6 @@ rtv_status pfail(rtv_prefill* p, rtv_status s, const std::string& msg) {
                    std::string(#call) + ": " + cudaGetErrorString(_e));                            \
   } while (0)
 
-struct DevGuard {
-  int prev = -1;
-  explicit DevGuard(int dev) {
-    cudaGetDevice(&prev);
-    if (prev != dev) cudaSetDevice(dev);
-  }
-  ~DevGuard() {
-    int cur = -1;
-    cudaGetDevice(&cur);
-    if (prev >= 0 && cur != prev) cudaSetDevice(prev);
-  }
-};
-
-int count_kernels(cudaGraph_t g) {
-  size_t n = 0;
-  if (cudaGraphGetNodes(g, nullptr, &n) != cudaSuccess) return -1;
-  std::vector<cudaGraphNode_t> nodes(n);
-  cudaGraphGetNodes(g, nodes.data(), &n);
-  int k = 0;
-  for (auto nd : nodes) {
-    cudaGraphNodeType t;
-    if (cudaGraphNodeGetType(nd, &t) == cudaSuccess && t == cudaGraphNodeTypeKernel) ++k;
-  }
-  return k;
-}
-
 void release(rtv_prefill::Entry& en) {
   if (en.ge.exec) cudaGraphExecDestroy(en.ge.exec);
   if (en.ge.graph) cudaGraphDestroy(en.ge.graph);
@@ -167,7 +141,7 @@ rtv_status get_entry(rtv_prefill* p, rtv_ctx* ex, int P, int n_steps, rtv_prefil
     if (s != RTV_OK) s = pfail(p, s, !blk->last_error.empty() ? blk->last_error : ex->last_error);
   }
   if (s == RTV_OK) {
-    en.ge.kernels = count_kernels(en.ge.graph);
+    en.ge.kernels = count_kernel_nodes(en.ge.graph);
     if (cudaStreamSynchronize(st) != cudaSuccess) s = pfail(p, RTV_ERR_CUDA, "prefill graph upload failed");
   }
   if (s != RTV_OK) {
@@ -233,7 +207,7 @@ rtv_status rtv_prefill_create(const rtv_prefill_config* cfg, int cuda_device, rt
   rtv_prefill* p = new rtv_prefill();
   p->cfg = c;
   p->device = cuda_device;
-  DevGuard dg(cuda_device);
+  DeviceGuard dg(cuda_device);
   rtv_status s = ctx_create(k, cuda_device, kGroup, true, &p->blk);
   if (s == RTV_OK && !p->blk->use_fast) s = RTV_ERR_UNSUPPORTED;
   if (s == RTV_OK) {
@@ -252,7 +226,7 @@ rtv_status rtv_prefill_load(rtv_prefill* p, const rtv_tensor* params, int n_para
   if (!p) return RTV_ERR_ARG;
   if (!params || n_params <= 0) return pfail(p, RTV_ERR_ARG, "no parameters");
   if (p->loaded) return pfail(p, RTV_ERR_STATE, "prefill stack already loaded");
-  DevGuard dg(p->device);
+  DeviceGuard dg(p->device);
   rtv_ctx* c = p->blk;
   c->W.layers.assign(c->cfg.n_layers, LayerW());
   SlotTable slots;
@@ -281,7 +255,7 @@ rtv_status rtv_prefill_kv(rtv_prefill* p, rtv_ctx* ex, const void* emb, int n_to
   if (!p) return RTV_ERR_ARG;
   rtv_status s = check_pair(p, ex, n_tokens);
   if (s != RTV_OK) return s;
-  DevGuard dg(p->device);
+  DeviceGuard dg(p->device);
   rtv_prefill::Entry* en = nullptr;
   s = get_entry(p, ex, n_tokens, 0, &en);
   if (s != RTV_OK) return s;
@@ -301,7 +275,7 @@ rtv_status rtv_prefill_denoise(rtv_prefill* p, rtv_ctx* ex, const void* emb, int
   if (!noise || !state || !actions_out) return pfail(p, RTV_ERR_ARG, "null pointer");
   if (n_steps <= 0 || n_steps > 64) return pfail(p, RTV_ERR_SHAPE, "n_steps must be in [1, 64]");
   if (ex->cfg.max_batch < 1) return pfail(p, RTV_ERR_SHAPE, "expert batch");
-  DevGuard dg(p->device);
+  DeviceGuard dg(p->device);
   rtv_prefill::Entry* en = nullptr;
   s = get_entry(p, ex, n_tokens, n_steps, &en);
   if (s != RTV_OK) return s;
@@ -334,7 +308,7 @@ int rtv_prefill_kernel_count(rtv_prefill* p, int n_tokens, int n_steps) {
 
 void rtv_prefill_destroy(rtv_prefill* p) {
   if (!p) return;
-  DevGuard dg(p->device);
+  DeviceGuard dg(p->device);
   cudaDeviceSynchronize();
   for (auto& kv : p->graphs) release(kv.second);
   for (void* q : p->allocs) cudaFree(q);

@@ -138,19 +138,6 @@ rtv_status dev_alloc_t(rtv_ctx* ctx, T** p, size_t count) {
     if (_s != RTV_OK) return _s;       \
   } while (0)
 
-struct DeviceGuard {
-  int prev = -1;
-  explicit DeviceGuard(int d) {
-    cudaGetDevice(&prev);
-    if (prev != d) cudaSetDevice(d);
-  }
-  ~DeviceGuard() {
-    int cur = -1;
-    cudaGetDevice(&cur);
-    if (prev >= 0 && cur != prev) cudaSetDevice(prev);
-  }
-};
-
 // SIMT forward of the expert over G suffixes (token rows T = G*S) and the
 // output head.  Used for the fp32 expert and, on request, the bf16 expert.
 template <typename WT>
@@ -171,19 +158,6 @@ void time_condition(rtv_ctx* ctx, const float* taus, int n, int n_steps, float* 
   launch_time_embedding(taus, n, n_steps, ctx->e_tmp, w, st);
   launch_linear<WT>(ctx->e_tmp, w, (const WT*)ctx->W.ti_w, ctx->W.ti_b, ctx->z_tmp, w, n, w, w, EPI_SWISH, st);
   launch_linear<WT>(ctx->z_tmp, w, (const WT*)ctx->W.to_w, ctx->W.to_b, c, w, n, w, w, EPI_STORE, st);
-}
-
-int count_kernel_nodes(cudaGraph_t g) {
-  size_t n = 0;
-  if (cudaGraphGetNodes(g, nullptr, &n) != cudaSuccess) return -1;
-  std::vector<cudaGraphNode_t> nodes(n);
-  cudaGraphGetNodes(g, nodes.data(), &n);
-  int k = 0;
-  for (auto nd : nodes) {
-    cudaGraphNodeType t;
-    if (cudaGraphNodeGetType(nd, &t) == cudaSuccess && t == cudaGraphNodeTypeKernel) ++k;
-  }
-  return k;
 }
 
 enum { KIND_DENOISE = 0, KIND_VERIFY = 1 };

@@ -61,6 +61,35 @@ struct ParamSlot {
 };
 using SlotTable = std::unordered_map<std::string, ParamSlot>;
 
+// Makes `dev` the current device for the guard's lifetime, then restores
+// the caller's device.
+struct DeviceGuard {
+  int prev = -1;
+  explicit DeviceGuard(int dev) {
+    cudaGetDevice(&prev);
+    if (prev != dev) cudaSetDevice(dev);
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    cudaGetDevice(&cur);
+    if (prev >= 0 && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+// Kernel nodes of a captured graph (-1 when the graph cannot be read).
+inline int count_kernel_nodes(cudaGraph_t g) {
+  size_t n = 0;
+  if (cudaGraphGetNodes(g, nullptr, &n) != cudaSuccess) return -1;
+  std::vector<cudaGraphNode_t> nodes(n);
+  cudaGraphGetNodes(g, nodes.data(), &n);
+  int k = 0;
+  for (auto nd : nodes) {
+    cudaGraphNodeType t;
+    if (cudaGraphNodeGetType(nd, &t) == cudaSuccess && t == cudaGraphNodeTypeKernel) ++k;
+  }
+  return k;
+}
+
 // Per-layer time modulation tables (RTV_TIME_ADARMS), rows of all layers:
 // mod [.][L][6w] = (scale_a, shift_a, gate_a, scale_m, shift_m, gate_m) of
 // every layer, sbq [.][L][Q+2KV] = W_qkv . shift_a and sbg [.][L][2F] =
