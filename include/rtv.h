@@ -268,7 +268,9 @@ rtv_status rtv_draft_create(const rtv_draft_config* cfg, int cuda_device, rtv_dr
  *   o_proj.w [w][Q]  mlp_norm.g [w]  gate_proj.w [F][w]  up_proj.w [F][w]
  *   down_proj.w [w][F]  action_head.w [A][w]  action_head.b [A]
  * Matrices in the config dtype, vectors in RTV_F32; every name exactly once.
- * Synchronous. */
+ * Synchronous.  A missing, duplicate or unknown name, or a wrong dtype
+ * returns RTV_ERR_ARG and a wrong shape RTV_ERR_SHAPE, before anything is
+ * allocated; a second load returns RTV_ERR_STATE. */
 rtv_status rtv_draft_load(rtv_draft* d, const rtv_tensor* params, int n_params);
 
 /* Candidate chunks chunk_out [batch][H][A] (fp32) from the image features
@@ -276,7 +278,10 @@ rtv_status rtv_draft_load(rtv_draft* d, const rtv_tensor* params, int n_params);
  * vis and chunk_out may be device or host memory (host copies are enqueued
  * on `stream`).  n_vis <= max_vis, batch <= max_batch.  Asynchronous; the
  * first call for a given (n_vis, batch) captures a CUDA graph (not on
- * `stream`), later calls replay it. */
+ * `stream`), later calls replay it.  Before rtv_draft_load: RTV_ERR_STATE;
+ * null pointers: RTV_ERR_ARG; sizes out of range: RTV_ERR_SHAPE; nothing is
+ * enqueued on an error.  Device-side errors go to the status word
+ * (rtv_draft_device_status). */
 rtv_status rtv_draft_forward(rtv_draft* d, const void* vis, int n_vis, int batch, float* chunk_out,
                              rtv_stream stream);
 
@@ -289,7 +294,11 @@ rtv_status rtv_draft_forward(rtv_draft* d, const void* vis, int n_vis, int batch
  * host memory *accepted_len, *flags (RTV_FLAG_*) and *used_full (1 = the
  * full path ran).  The expert's prefix KV must be installed with batch 1;
  * its chunk_len and action_dim must equal the draft's n_queries and
- * action_dim.  Synchronous: returns once actions_out holds the chunk. */
+ * action_dim.  Synchronous: returns once actions_out holds the chunk.
+ * Errors: null pointers or a draft on another device RTV_ERR_ARG, shape
+ * mismatches or a prefix of batch > 1 RTV_ERR_SHAPE, and whatever
+ * rtv_draft_forward, rtv_verify or rtv_denoise return (their message is
+ * copied to rtv_draft_last_error). */
 rtv_status rtv_flash_round(rtv_ctx* ctx, rtv_draft* d, const void* vis, int n_vis, const float* noise,
                            const float* state, const float* taus, int n_taus, float delta, int gripper_dim,
                            int n_steps, float* actions_out, int* accepted_len, unsigned* flags, int* used_full,
@@ -342,7 +351,8 @@ rtv_status rtv_prefill_create(const rtv_prefill_config* cfg, int cuda_device, rt
 
 /* Copy and pack the stack's parameters: for every layer l the names of
  * rtv_load_expert's layers (layers.l.attn_norm.g, layers.l.q_proj.w, ...,
- * layers.l.down_proj.w), matrices in bf16, gains in RTV_F32.  Synchronous. */
+ * layers.l.down_proj.w), matrices in bf16, gains in RTV_F32.  Synchronous.
+ * Name, dtype and shape errors as for rtv_draft_load. */
 rtv_status rtv_prefill_load(rtv_prefill* p, const rtv_tensor* params, int n_params);
 
 /* Run the stack over emb [n_tokens][width] (bf16, device or host) and
@@ -350,7 +360,10 @@ rtv_status rtv_prefill_load(rtv_prefill* p, const rtv_tensor* params, int n_para
  * prefix_len = n_tokens), as rtv_set_prefix_kv would.  The expert must be a
  * bf16 tensor-core context with the stack's n_layers, n_kv_heads and
  * head_dim, and n_tokens <= its max_prefix_len.  Asynchronous on `stream`;
- * the first call for a given n_tokens captures a CUDA graph. */
+ * the first call for a given n_tokens captures a CUDA graph.  Before both
+ * loads: RTV_ERR_STATE; a mismatched expert or n_tokens out of range:
+ * RTV_ERR_SHAPE; an expert off the tensor-core path: RTV_ERR_UNSUPPORTED;
+ * nothing is enqueued on an error. */
 rtv_status rtv_prefill_kv(rtv_prefill* p, rtv_ctx* ctx, const void* emb, int n_tokens, rtv_stream stream);
 
 /* Prefill followed by rtv_denoise(ctx, noise, state, n_steps) for one
