@@ -402,3 +402,40 @@ def test_fp8_mlp_weights_within_the_format_bound():
         rows = np.arange(draw.shape[0])
         amax_idx = np.argmax(np.abs(draw), axis=1)
         assert np.allclose(W[key][rows, amax_idx], draw[rows, amax_idx], rtol=1e-6, atol=0)
+
+
+# ---------------------------------------------------------------------------
+# structure of the batched verification, and the GEMM primitive
+# ---------------------------------------------------------------------------
+
+def test_batched_verify_equals_separate_single_tau_calls():
+    """Verification at several taus is the taus one at a time: the distance
+    row of tau_i does not depend on the other taus, and the accepted length
+    is the shortest of the single-tau lengths."""
+    cfg = tiny()
+    W = tiny_weights(cfg, seed=7)
+    kv = make_prefix_kv(cfg, seed=7)
+    state = make_state(cfg, seed=7)[0]
+    draft = make_draft(cfg, seed=7)
+    eps = make_noise(cfg, seed=7)[0]
+    taus = (0.2, 0.5, 0.8)
+    n_acc, _, dist = O.verify(W, cfg, draft, eps, state, kv, taus, 0.4, cfg.gripper)
+    singles = [O.verify(W, cfg, draft, eps, state, kv, (t,), 0.4, cfg.gripper) for t in taus]
+    for i, (_, _, d1) in enumerate(singles):
+        np.testing.assert_array_equal(dist[i], d1[0])
+    assert n_acc == min(s[0] for s in singles)
+
+
+def test_linear_matches_a_naive_triple_loop():
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((3, 5))
+    w = rng.standard_normal((4, 5))
+    b = rng.standard_normal(4)
+    y = np.zeros((3, 4))
+    for i in range(3):
+        for j in range(4):
+            acc = 0.0
+            for k in range(5):
+                acc += x[i, k] * w[j, k]
+            y[i, j] = acc + b[j]
+    np.testing.assert_allclose(O.linear(x, w, b), y, rtol=1e-14, atol=1e-14)
