@@ -384,7 +384,11 @@ const char* rtv_prefill_last_error(rtv_prefill* p);
  * is rtv_prefill_kv's graph.  -1 before it has been captured. */
 int rtv_prefill_kernel_count(rtv_prefill* p, int n_tokens, int n_steps);
 
-/* Release every resource of the prefill stack.  NULL is accepted. */
+/* Release every resource of the prefill stack.  NULL is accepted.  The
+ * stack keeps the graphs it captured for an expert context (they address
+ * that context's buffers): destroy the stack before, or together with, every
+ * expert it has served, and do not pass it a context created after one of
+ * those was destroyed. */
 void rtv_prefill_destroy(rtv_prefill* p);
 
 #ifdef __cplusplus
