@@ -172,8 +172,22 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def oracle_step_seconds(cfg, target_s: float, min_samples: int = 1, max_samples: int = 10):
-    """Seconds per Euler step of the CPU oracle on the workload (bounded sample)."""
+def oracle_step_seconds_threads(cfg, target_s: float, threads=None, min_samples: int = 5, max_samples: int = 10):
+    """oracle_step_seconds with the BLAS thread pool limited to `threads`
+    (None: as configured, i.e. every host core)."""
+    if threads is None:
+        return oracle_step_seconds(cfg, target_s, min_samples, max_samples)
+    try:
+        from threadpoolctl import threadpool_limits
+    except Exception:
+        return None, 0
+    with threadpool_limits(limits=threads, user_api="blas"):
+        return oracle_step_seconds(cfg, target_s, min_samples, max_samples)
+
+
+def oracle_step_seconds(cfg, target_s: float, min_samples: int = 5, max_samples: int = 10):
+    """Seconds per Euler step of the CPU oracle on the workload (bounded
+    sample: median of at least min_samples steps)."""
     from oracle import expert as O
     from synthetic import make_noise, make_prefix_kv, make_state, make_weights
     W = O.to_f64(make_weights(cfg))
@@ -294,14 +308,18 @@ def run_reference(args, info):
     per_step = (time.perf_counter() - t0) / steps
     chunk_us = per_step * cfg.n_steps * 1e6
     cores = blas_threads()
+    # one timed step is one Euler step of the chunk: steps x ms_per_step is the
+    # time actually spent; value is that per-step time scaled to a whole chunk
     line = {
         "impl": "reference", "metric": METRIC, "value": chunk_us, "unit": "us", "n_gpus": args.gpus,
-        "steps": steps, "warmup": args.warmup, "ms_per_step": chunk_us / 1000.0, "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "n_steps": cfg.n_steps, "batch": 1, "prefix_len": cfg.prefix_len},
+        "steps": steps, "warmup": min(args.warmup, 1), "ms_per_step": per_step * 1000.0,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "n_steps": cfg.n_steps, "batch": 1, "prefix_len": cfg.prefix_len,
+                   "layers": cfg.n_layers, "width": cfg.width, "path": "cpu oracle (fp64 numpy)",
+                   "step": f"one Euler step of the chunk; value = ms_per_step x {cfg.n_steps} (chunk latency)"},
         "cpu_baseline": {"value": chunk_us, "unit": "us", "cores": cores, "kind": "oracle",
                          "sample": f"{steps} single Euler steps of the {args.workload} chunk (fp64 numpy oracle), "
-                                   f"each scaled x{cfg.n_steps} to chunk latency"},
+                                   f"mean scaled x{cfg.n_steps} to chunk latency"},
         "e2e": {"value": chunk_us, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -371,6 +389,22 @@ def run_ours(args, info):
     s, bits = ex.status()
     if s != 0:
         raise RuntimeError(f"device status {bits:#x} after the timed region")
+
+    # latency distribution: each call bracketed by its own events and waited
+    # for (no overlap between calls), at least 50 calls
+    lat = []
+    for _ in range(max(50, K)):
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        ex.denoise(noise_d, state_d, n, out_d, stream=stream)
+        c1.record(stream)
+        c1.synchronize()
+        lat.append(c0.elapsed_time(c1) * 1000.0)
+    lat = np.asarray(lat)
+    latency = {"unit": "us", "calls": int(lat.size), "p50": float(np.percentile(lat, 50)),
+               "p90": float(np.percentile(lat, 90)), "p99": float(np.percentile(lat, 99)),
+               "mean": float(lat.mean()), "min": float(lat.min()), "max": float(lat.max()),
+               "note": "per-call CUDA events on the launching stream, each call waited for before the next"}
 
     # end to end through the C ABI with pinned host buffers
     noise_h = torch.from_numpy(noise).pin_memory()
@@ -452,6 +486,7 @@ def run_ours(args, info):
                                      "allow and 18 do not)"},
         "e2e": {"value": e2e_ms * 1000.0, "unit": "us",
                 "h2d_bytes_per_step": int(noise.nbytes + state.nbytes), "d2h_bytes_per_step": int(noise.nbytes)},
+        "latency": latency,
         "clocks": clk.summary(),
         "gpu_launches": int(launches_per_call * K) if launches_per_call > 0 else None,
         "verify": {"taus": list(taus), "us_per_call": verify_us,
@@ -462,11 +497,16 @@ def run_ours(args, info):
     if round_info is not None:
         line["flash_round"] = round_info
     if info.world == 1 and not args.no_cpu_baseline:
-        per_step_s, k = oracle_step_seconds(cfg, args.cpu_seconds)
+        per_step_s, k = oracle_step_seconds_threads(cfg, args.cpu_seconds)
         line["cpu_baseline"] = {
             "value": per_step_s * n * 1e6, "unit": "us", "cores": blas_threads(), "kind": "oracle",
             "sample": f"{k} single Euler steps of the {args.workload} chunk (fp64 numpy oracle, median), "
-                      f"scaled x{n} to one chunk"}
+                      f"scaled x{n} to one chunk; BLAS threads = host cores"}
+        one_s, k1 = oracle_step_seconds_threads(cfg, args.cpu_seconds / 2, threads=1)
+        if one_s is not None:
+            line["cpu_baseline"]["single_thread"] = {
+                "value": one_s * n * 1e6, "unit": "us", "cores": 1,
+                "sample": f"{k1} single Euler steps, median, scaled x{n}; BLAS limited to one thread"}
     print(json.dumps(line), flush=True)
 
 

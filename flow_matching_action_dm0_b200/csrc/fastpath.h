@@ -53,6 +53,13 @@ rtv_status fast_block_embed(rtv_ctx* ctx, const float* rows, int n_src_rows, int
 rtv_status fast_prefill(rtv_ctx* pre, rtv_ctx* ex, const __nv_bfloat16* emb, int P, const float* rope_cs,
                         const float* rope_sn, cudaStream_t st);
 void fast_destroy(rtv_ctx* ctx);
+// Read-only view of the tensor-core layouts another kernel family reuses
+// (packed weights, transposed embeddings, prefix tiles); false without them.
+struct FastViews {
+  const __nv_bfloat16 *w_qkv, *w_o, *w_gu, *w_down, *w_aiT, *w_spT, *pkt, *pvt;
+  int ntile_max, num_sms;
+};
+bool fast_views(const rtv_ctx* ctx, FastViews* out);
 // Diagnostic phase trace (only when the RTV_TRACE environment variable is set).
 void fast_arm_trace(rtv_ctx* ctx);
 void fast_trace_report(rtv_ctx* ctx);

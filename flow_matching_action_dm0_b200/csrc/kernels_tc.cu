@@ -2440,6 +2440,23 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
   return RTV_OK;
 }
 
+bool fast_views(const rtv_ctx* ctx, FastViews* out) {
+  const FastPath* fp = ctx->fast;
+  // (the packed weights exist only after rtv_load_expert; callers check them before use)
+  if (!fp || !fp->tc_attn || !fp->pkt || ctx->cfg.mlp_dtype == RTV_FP8_E4M3) return false;
+  out->w_qkv = fp->w_qkv;
+  out->w_o = fp->w_o;
+  out->w_gu = fp->w_gu;
+  out->w_down = fp->w_down;
+  out->w_aiT = fp->w_aiT;
+  out->w_spT = fp->w_spT;
+  out->pkt = fp->pkt;
+  out->pvt = fp->pvt;
+  out->ntile_max = fp->ntile_max;
+  out->num_sms = fp->num_sms;
+  return true;
+}
+
 void fast_destroy(rtv_ctx* ctx) {
   if (!ctx->fast) return;
   for (void* p : ctx->fast->allocs) cudaFree(p);

@@ -11,8 +11,12 @@
 // The staging array is shared by every context and every call on a device,
 // and it keeps whatever the last call left in it.  Calls whose work overlaps
 // on the GPU (different streams, or different contexts on one device) race
-// on it: serialise them.  Every GPU that loads this library holds the array
-// (kStageBytes) until the process exits.
+// on it: serialise them.  The array (kStageBytes) lives in this file's
+// module.  CUDA loads modules lazily, so the first call on a device -- which
+// looks up the array's device address -- may be the moment the driver loads
+// the module and reserves the array; that first call should therefore come
+// at set-up time, before any stream capture.  From then on the device holds
+// the array until the process exits and no call allocates anything.
 #include <mutex>
 #include <string>
 
@@ -83,15 +87,27 @@ extern "C" rtv_status rtv_set_prefix_kv_static(rtv_ctx* ctx, const void* kv, int
   rtv_status s = stage_address(ctx, &stage);
   cudaStream_t st = (cudaStream_t)stream;
   cudaPointerAttributes at{};
-  const bool on_device = cudaPointerGetAttributes(&at, kv) == cudaSuccess && at.type == cudaMemoryTypeDevice;
+  const bool dev_mem = cudaPointerGetAttributes(&at, kv) == cudaSuccess && at.type == cudaMemoryTypeDevice;
   cudaGetLastError();
+  // Device memory of this GPU is read in place by the pack kernel; another
+  // GPU's memory is refused (the pack kernel would need peer access to it).
+  if (s == RTV_OK && dev_mem && at.device != ctx->device) {
+    ctx->last_error = "prefix kv is device memory of another GPU (" + std::to_string(at.device) + ")";
+    s = RTV_ERR_ARG;
+  }
+  const bool on_device = dev_mem;
+  // From here on the library's cache is being overwritten: until every layer
+  // is installed, denoise and verify refuse to run (RTV_ERR_STATE) rather
+  // than read a cache that mixes two prefixes.
+  if (s == RTV_OK) ctx->have_prefix = false;
   const size_t dst_layer = (size_t)2 * k.max_batch * k.n_kv_heads * k.max_prefix_len * k.head_dim;
   for (int l = 0; l < k.n_layers && s == RTV_OK; ++l) {
     const char* src = (const char*)kv + (size_t)l * bytes_layer;
     if (!on_device) {
-      // host data goes through the staging array; the pack below reads it
-      // before the next layer's copy overwrites it (same stream)
-      const cudaError_t e = cudaMemcpyAsync(stage, src, bytes_layer, cudaMemcpyHostToDevice, st);
+      // host (pageable or pinned) or managed data goes through the staging
+      // array; the pack below reads it before the next layer's copy
+      // overwrites it (same stream)
+      const cudaError_t e = cudaMemcpyAsync(stage, src, bytes_layer, cudaMemcpyDefault, st);
       if (e != cudaSuccess) {
         ctx->last_error = std::string("cudaMemcpyAsync to the staging array: ") + cudaGetErrorString(e);
         s = RTV_ERR_CUDA;

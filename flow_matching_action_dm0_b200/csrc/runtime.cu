@@ -14,6 +14,7 @@
 
 #include "fastpath.h"
 #include "kernels.h"
+#include "resident.h"
 #include "runtime.h"
 
 using namespace rtv;
@@ -206,6 +207,10 @@ rtv_status build_graph(rtv_ctx* ctx, int kind, int n, int batch, int P, GraphEnt
   }
   CK(cudaGetLastError());
   CK(cudaStreamSynchronize(st));
+  // The resident kernel serves the plain time condition on the tensor-core
+  // path when its plan fits (prepared here, outside the capture).
+  const bool use_res = ctx->use_fast && tc == RTV_TIME_ADD &&
+                       resident_prepare(ctx, kind == KIND_DENOISE ? batch : n, P, kind == KIND_VERIFY);
 
   if (ctx->use_fast) fast_arm_trace(ctx);
   CK(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
@@ -226,7 +231,9 @@ rtv_status build_graph(rtv_ctx* ctx, int kind, int n, int batch, int P, GraphEnt
       m.group_rows = 0;
       return m;
     };
-    if (ctx->use_fast) {
+    if (use_res) {
+      chain(resident_launch(ctx, batch, P, n, false, ctab, cs, sn, st));
+    } else if (ctx->use_fast) {
       // step boundary k: head of step k-1 (k > 0) and embedding of step k (k < n)
       auto embed_tail = [&](int step) {
         if (tc == RTV_TIME_CONCAT) {
@@ -280,7 +287,9 @@ rtv_status build_graph(rtv_ctx* ctx, int kind, int n, int batch, int P, GraphEnt
       m.group_rows = 1;
     }
     const ModTables* mp = tc == RTV_TIME_ADARMS ? &m : nullptr;
-    if (ctx->use_fast) {
+    if (use_res) {
+      chain(resident_launch(ctx, T, P, 1, true, ctx->c_verify, cs, sn, st));
+    } else if (ctx->use_fast) {
       chain(fast_step(ctx, T, false, true, 0.f, add_c ? ctx->c_verify : ctx->czero, add_c ? w : 0, 0, false, st,
                       mp ? ctx->mod_v : nullptr, mp ? L * 6 * w : 0));
       if (tc == RTV_TIME_CONCAT) {
@@ -420,6 +429,7 @@ rtv_status ctx_create(const rtv_expert_config& k, int cuda_device, int S, bool b
     const char* env = getenv("RTV_PATH");
     const bool want_simt = env && strcmp(env, "simt") == 0;
     if (!want_simt) s = fast_create(ctx);
+    if (s == RTV_OK && ctx->use_fast) s = resident_create(ctx);
   }
   if (s == RTV_OK && k.mlp_dtype == RTV_FP8_E4M3 && !ctx->use_fast) s = RTV_ERR_UNSUPPORTED;   // no SIMT FP8
   if (s != RTV_OK) {
@@ -573,6 +583,7 @@ rtv_status rtv_load_expert(rtv_ctx* ctx, const rtv_tensor* params, int n_params)
     add_layer_slots(ctx, slots, "layers." + std::to_string(l) + ".", W.layers[l]);
   TRY(load_slots(ctx, slots, params, n_params));
   if (ctx->use_fast) TRY(fast_load(ctx, params, n_params));
+  TRY(resident_load(ctx));
   CK(cudaDeviceSynchronize());
   ctx->loaded = true;
   return RTV_OK;
@@ -634,7 +645,10 @@ rtv_status rtv_denoise(rtv_ctx* ctx, const float* noise, const float* state, int
   CK(cudaMemcpyAsync(ctx->state, state, (size_t)B * k.state_dim * sizeof(float), cudaMemcpyDefault, st));
   CK(cudaGraphLaunch(ge->exec, st));
   CK(cudaMemcpyAsync(actions_out, ctx->x, xb, cudaMemcpyDefault, st));
-  if (ctx->use_fast && getenv("RTV_TRACE")) fast_trace_report(ctx);
+  if (ctx->use_fast && getenv("RTV_TRACE")) {
+    fast_trace_report(ctx);
+    resident_trace_report(ctx);
+  }
   return RTV_OK;
 }
 
@@ -668,7 +682,10 @@ rtv_status rtv_verify(rtv_ctx* ctx, const float* draft, const float* noise, cons
   CK(cudaMemcpyAsync(accepted_len, ctx->accepted, sizeof(int), cudaMemcpyDefault, st));
   CK(cudaMemcpyAsync(flags, ctx->flags, sizeof(unsigned), cudaMemcpyDefault, st));
   if (dist) CK(cudaMemcpyAsync(dist, ctx->dist, (size_t)n_taus * ctx->H * sizeof(float), cudaMemcpyDefault, st));
-  if (ctx->use_fast && getenv("RTV_TRACE")) fast_trace_report(ctx);
+  if (ctx->use_fast && getenv("RTV_TRACE")) {
+    fast_trace_report(ctx);
+    resident_trace_report(ctx);
+  }
   return RTV_OK;
 }
 
@@ -706,6 +723,7 @@ void rtv_destroy(rtv_ctx* ctx) {
     if (kv.second.graph) cudaGraphDestroy(kv.second.graph);
     for (void* p : kv.second.owned) cudaFree(p);
   }
+  if (ctx->resident) resident_destroy(ctx);
   if (ctx->fast) fast_destroy(ctx);
   for (void* p : ctx->allocs) cudaFree(p);
   if (ctx->cap_stream) cudaStreamDestroy(ctx->cap_stream);

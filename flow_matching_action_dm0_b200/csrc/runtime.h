@@ -47,6 +47,7 @@ struct GraphEntry {
 };
 
 struct FastPath;  // tensor-core path state (kernels_tc.cu)
+struct ResidentState;  // resident-kernel state (resident.cu)
 
 // One named parameter of a load table: expected shape and dtype, and where it
 // goes (its own allocation, or an offset inside a packed allocation).
@@ -144,6 +145,7 @@ struct rtv_ctx {
   std::map<std::tuple<int, int, int, int>, rtv::GraphEntry> graphs;  // (kind, n, batch/taus, prefix_len)
 
   rtv::FastPath* fast = nullptr;
+  rtv::ResidentState* resident = nullptr;   // set when the resident kernel serves this context's shapes
 };
 
 namespace rtv {

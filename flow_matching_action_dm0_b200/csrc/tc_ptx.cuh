@@ -1,5 +1,5 @@
 // Thin wrappers over the sm_100a PTX used by the tensor-core kernels:
-// mbarriers, TMA tile loads, tcgen05 (UMMA) issue / commit / TMEM access,
+// mbarriers, bulk copies, tcgen05 (UMMA) issue / commit / TMEM access,
 // cluster barriers and distributed shared memory, programmatic dependent
 // launch, and the legacy warp-level mma.sync / ldmatrix used by attention.
 #pragma once
@@ -54,28 +54,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
   }
 }
 
-// ---- TMA --------------------------------------------------------------------
+// ---- bulk copies ----------------------------------------------------------------
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
-}
-// 2-D tiled load of a box into shared memory; completion counted on `bar` in bytes.
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
-                                            uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
-      : "memory");
-}
-// Same without an L2 cache-policy operand.
-__device__ __forceinline__ void tma_load_2d_nohint(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
-      : "memory");
 }
 // Contiguous copy of `bytes` (a multiple of 16; both addresses 16-byte
 // aligned) from global to shared memory; completion counted on `bar` in bytes.
@@ -97,9 +80,6 @@ __device__ __forceinline__ void bulk_load_hint(void* dst, const void* src, uint3
 // Hint: bring `bytes` (a multiple of 16) of global memory into L2.
 __device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
-  asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 

@@ -177,12 +177,18 @@ rtv_status rtv_set_prefix_kv(rtv_ctx* ctx, const void* kv, int prefix_len, int b
  * through a fixed 4 MiB array in device global memory that the library
  * declares statically (every GPU that loads the library holds it until the
  * process exits).  Returns RTV_ERR_SHAPE when one layer's keys and values
- * (2 * batch * prefix_len * n_kv_heads * head_dim elements) exceed 4 MiB.
- * The first call on a device looks up the array's device address; make that
- * first call before any stream capture.  All calls share the array and it
- * keeps the last call's contents: calls whose work overlaps on the GPU (other
- * streams or other contexts on the same device) race on it, so serialise
- * them.  Calls no cudaMalloc, cudaFree or allocating library routine. */
+ * (2 * batch * prefix_len * n_kv_heads * head_dim elements) exceed 4 MiB,
+ * and RTV_ERR_ARG for device memory of another GPU (device memory of the
+ * context's GPU is read in place; host and managed memory are staged).
+ * The first call on a device looks up the array's device address, which may
+ * make the driver load the library's module and reserve the array then
+ * (lazy module loading): make that first call at set-up time, before any
+ * stream capture.  All calls share the array and it keeps the last call's
+ * contents: calls whose work overlaps on the GPU (other streams or other
+ * contexts on the same device) race on it, so serialise them.  While the
+ * copy runs the context holds no prefix: if the call fails part-way,
+ * denoise and verify return RTV_ERR_STATE until a prefix is installed.
+ * Calls no cudaMalloc, cudaFree or allocating library routine. */
 rtv_status rtv_set_prefix_kv_static(rtv_ctx* ctx, const void* kv, int prefix_len, int batch, rtv_stream stream);
 
 /* Denoise ([DM0.5] 5.3): from noise x_1 = noise [batch][H][A], run n_steps

@@ -123,14 +123,23 @@ def test_pi0_bf16_batch_sixteen_token_tiles(cuda_ok):
     assert bf16_tolerance_ok(got, ref), (rel_l2(got, ref), np.max(np.abs(got - ref)))
 
 
-def test_repeat_calls_are_bitwise_identical(cuda_ok):
+@pytest.mark.parametrize("path", ["layered", "default"])
+def test_repeat_calls_agree(cuda_ok, monkeypatch, path):
+    """The layered kernels reduce split-K partial sums in a fixed rank order:
+    repeated calls are bit-for-bit equal.  The resident kernel adds them in
+    L2 in the order they arrive: repeated calls agree to fp32 rounding."""
+    if path == "layered":
+        monkeypatch.setenv("RTV_PATH", "layered")
     cfg = get_config("pi0-bf16", n_layers=2)
     ex, _, _ = build_expert(cfg)
     noise, state = make_noise(cfg), make_state(cfg)
     a = ex.denoise(noise, state, 5)
     b = ex.denoise(noise, state, 5)
     ex.close()
-    np.testing.assert_array_equal(a, b)
+    if path == "layered":
+        np.testing.assert_array_equal(a, b)
+    else:
+        assert rel_l2(b, a) <= 1e-5, rel_l2(b, a)
 
 
 def test_simt_path_on_bf16_expert_matches_oracle(cuda_ok, monkeypatch):

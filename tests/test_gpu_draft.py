@@ -178,8 +178,12 @@ def test_full_size_round_is_consistent(cuda_ok):
         acc, flags, _ = ex.verify(draft, eps, state, cfg.taus, delta, cfg.gripper)
         assert (r.accepted_len, r.flags) == (acc, flags)
         assert r.used_full == bool(flags & (O.FLAG_ZERO_ACCEPT | O.FLAG_SWITCH))
-        expect = ex.denoise(eps[None], state[None], 10)[0] if r.used_full else draft
-        np.testing.assert_array_equal(r.chunk, expect)
+        if r.used_full:
+            # the denoised chunk from the same noise (fp32 sums in arrival order: equal to rounding)
+            expect = ex.denoise(eps[None], state[None], 10)[0]
+            assert rel_l2(r.chunk, expect) <= 1e-5
+        else:
+            np.testing.assert_array_equal(r.chunk, draft)
     s, bits = dm.status()
     assert s == 0 and bits == 0
     dm.close()

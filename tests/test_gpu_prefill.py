@@ -71,7 +71,7 @@ def test_prefill_denoise_matches_oracle_small(cuda_ok, n_tokens):
     # rtv_denoise gives the same chunk as the one-graph call
     pf.kv(ex, emb)
     again = ex.denoise(noise, state, 3)[0]
-    np.testing.assert_array_equal(again, got)
+    assert rel_l2(again, got) <= 1e-5, rel_l2(again, got)
     pf.close()
     ex.close()
 

@@ -59,14 +59,19 @@ def test_tiny_fp32_verify_matches_oracle(cuda_ok, n_switch):
     assert bool(got[1] & 2) == bool(n_switch)
 
 
-def test_pi0_verify_three_taus_matches_oracle(cuda_ok):
+@pytest.mark.parametrize("n_switch", [0, 1])
+def test_pi0_verify_three_taus_matches_oracle(cuda_ok, n_switch):
+    # the draft of the FLASH verification workload has 0 or 1 gripper sign switch:
+    # without one the fallback flag comes from the accepted length alone
     cfg = get_config("pi0-verify")
-    ex, got, ref, (draft, _, _, delta) = run_verify(cfg, cfg.taus, n_switch=1)
+    ex, got, ref, (draft, _, _, delta) = run_verify(cfg, cfg.taus, n_switch=n_switch)
     ex.close()
-    print("pi0-verify rel_l2(dist) =", rel_l2(got[2], ref[2]), "accepted", got[0], ref[0], "delta", delta)
+    print("pi0-verify n_switch", n_switch, "rel_l2(dist) =", rel_l2(got[2], ref[2]), "accepted", got[0], ref[0],
+          "delta", delta)
     assert rel_l2(got[2], ref[2]) <= 1e-2
     assert np.max(np.abs(got[2] - ref[2])) <= 3e-2
     assert got[0] == ref[0] and got[1] == ref[1]
+    assert bool(got[1] & 2) == bool(n_switch)
 
 
 def test_decision_rule_on_device_distances_is_bit_exact(cuda_ok):
@@ -77,8 +82,10 @@ def test_decision_rule_on_device_distances_is_bit_exact(cuda_ok):
     cands = [0.0, float(dist.max()) * 2, float(dist[1, 3]), float(np.nextafter(np.float32(dist[0, 5]), np.inf)),
              float(np.median(dist))]
     for delta in cands:
+        # the decision of a call is the rule applied to that call's own distances
+        # (repeated calls agree to fp32 rounding, not bit for bit)
         acc, flags, d2 = ex.verify(draft, eps, state, (0.2, 0.5, 0.8), delta, cfg.gripper)
-        np.testing.assert_array_equal(d2, dist)
+        assert rel_l2(d2, dist) <= 1e-5
         assert (acc, flags) == O.verify_decide(d2, draft, delta, cfg.gripper)
     ex.close()
 
