@@ -341,6 +341,7 @@ __global__ void __launch_bounds__(kRThreads, 1) resident_kernel(const ResArgs a)
   __shared__ float s_red[2][128];    // attention: per-row halves (max, then sum)
   __shared__ float s_wred[8];
   __shared__ int s_gr[128];          // attention: global row index of each tile row (-1: padding)
+  __shared__ unsigned s_brk[4];      // attention: rows where a run of consecutive global rows breaks
   const int cta = blockIdx.x, ncta = gridDim.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int* pl = a.plan + (size_t)cta * kPlanInts;
@@ -966,6 +967,12 @@ __global__ void __launch_bounds__(kRThreads, 1) resident_kernel(const ResArgs a)
       const int n_keys = pre ? min(64, a.P - 64 * kt) : a.S;
       const int n_vis = (!pre && a.mask_mode == RTV_MASK_PI0_BLOCK && rr.s == 0) ? 1 : n_keys;
       if (workers_any(*abort)) return false;
+      // row r starts a new run of consecutive global rows (or is past the valid rows)
+      if (half == 0) {
+        const bool brk = r > 0 && (!row_valid || s_gr[r] != s_gr[r - 1] + 1);
+        const unsigned m = __ballot_sync(0xffffffffu, brk);
+        if (lane == 0) s_brk[quarter] = m;
+      }
       const bool s_done = mwait(&ctl.att_s, att_no & 1, a.timeout_ns, abort);
       if (!s_done && !*abort) raise_abort(a, &ctl, true);
       if (workers_any(!s_done)) return false;
@@ -1042,11 +1049,18 @@ __global__ void __launch_bounds__(kRThreads, 1) resident_kernel(const ResArgs a)
         ptx::fence_proxy_async_smem();
         workers_sync();
         if (wt == 0) {
-          // rows whose global indices are consecutive go in one operation
+          // rows whose global indices are consecutive go in one operation: the
+          // runs start where the ballots below marked a break
           int i0 = 0;
           while (i0 < n_rows) {
-            int i1 = i0 + 1;
-            while (i1 < n_rows && s_gr[i1] == s_gr[i1 - 1] + 1) ++i1;
+            int i1 = n_rows;
+            for (int q = (i0 + 1) >> 5; q < 4 && q * 32 < n_rows; ++q) {
+              const unsigned m = s_brk[q] & (q == ((i0 + 1) >> 5) ? ~((1u << ((i0 + 1) & 31)) - 1u) : ~0u);
+              if (m) {
+                i1 = min(n_rows, q * 32 + __ffs(m) - 1);
+                break;
+              }
+            }
             bulk_store(dst_slot + ((size_t)cb * a.R_att + s_gr[i0]) * 64, ptx::smem_u32(stg + i0 * 64),
                        (uint32_t)((i1 - i0) * 256));
             i0 = i1;

@@ -64,13 +64,20 @@ def test_resident_batch_two_matches_oracle(cuda_ok, resident):
 
 
 def test_resident_repeat_calls_agree_to_rounding(cuda_ok, resident):
+    """The split-K sums meet in arrival order: the last bits of a sum differ
+    between calls, and through the bf16 roundings of every operand that
+    follows, the two calls' rounding noise decorrelates.  Repeated calls then
+    differ at the bf16 level (not more), and each stays within the oracle's
+    tolerance."""
     cfg = get_config("pi0-bf16", n_layers=2)
-    ex, _, _ = build_expert(cfg)
+    ex, weights, kv = build_expert(cfg)
     noise, state = make_noise(cfg), make_state(cfg)
     a = ex.denoise(noise, state, 5)
     b = ex.denoise(noise, state, 5)
     ex.close()
-    assert rel_l2(b, a) <= 1e-5, rel_l2(b, a)
+    ref = O.denoise(O.to_f64(weights), cfg, noise, state, kv, 5)
+    assert bf16_tolerance_ok(b, a), rel_l2(b, a)
+    assert bf16_tolerance_ok(a, ref) and bf16_tolerance_ok(b, ref)
 
 
 @pytest.mark.parametrize("n_switch", [0, 1])
