@@ -26,7 +26,7 @@ _TIME = {"add": L.RTV_TIME_ADD, "concat": L.RTV_TIME_CONCAT, "adarms": L.RTV_TIM
 
 
 def make_config(shape, max_batch: Optional[int] = None, max_taus: int = 4,
-                max_prefix_len: Optional[int] = None) -> L.rtv_expert_config:
+                max_prefix_len: Optional[int] = None, barrier_timeout_ns: int = 0) -> L.rtv_expert_config:
     g = lambda n, d=None: getattr(shape, n, d)  # noqa: E731
     cfg = L.rtv_expert_config()
     for n in ("n_layers", "width", "n_q_heads", "n_kv_heads", "head_dim", "mlp_dim", "action_dim", "state_dim",
@@ -40,7 +40,7 @@ def make_config(shape, max_batch: Optional[int] = None, max_taus: int = 4,
     cfg.suffix_mask = _MASKS[g("suffix_mask", "bidir")]
     cfg.rms_eps = float(g("rms_eps", 1e-6))
     cfg.rope_theta = float(g("rope_theta", 10000.0))
-    cfg.barrier_timeout_ns = 0
+    cfg.barrier_timeout_ns = int(barrier_timeout_ns)   # 0: the library's default limit
     cfg.time_cond = _TIME[g("time_cond", "add")]
     return cfg
 
@@ -119,9 +119,9 @@ def make_tensors(weights: Dict[str, object], matrix_dtype: int, overrides: Optio
 
 class ActionExpert:
     def __init__(self, shape, device: int = 0, max_batch: Optional[int] = None, max_taus: int = 4,
-                 max_prefix_len: Optional[int] = None):
+                 max_prefix_len: Optional[int] = None, barrier_timeout_ns: int = 0):
         self.shape = shape
-        self.cfg = make_config(shape, max_batch, max_taus, max_prefix_len)
+        self.cfg = make_config(shape, max_batch, max_taus, max_prefix_len, barrier_timeout_ns)
         self.device = device
         self.h = L.rtv_create(self.cfg, device)
         self._keep = []
