@@ -165,9 +165,15 @@ __host__ __device__ inline GemmSmem gemm_smem_layout(int stages, int n_mma, int 
     s.in_off = s.recv_off + cs * per * 512;   // [per][128] fp32 epilogue inputs of the owned tokens
   }
   s.bar_off = s.in_off + (with_in ? per * 512 : 0);   // GU reads no per-token epilogue inputs
-  s.total = s.bar_off + (3 * stages + 2) * 8 + 16 + 1024;   // barriers, TMEM slot, alignment slack
+  s.total = s.bar_off + (4 * stages + 2) * 8 + 16 + 1024;   // barriers, TMEM slot, alignment slack
   return s;
 }
+
+// Limit of the waits that only drain work this CTA has already issued
+// (copies and MMAs that complete without help from any other agent): after a
+// timeout a CTA stops issuing, then waits this long at most for what is still
+// in flight before it leaves.
+constexpr long long kDrainNs = 200000000ll;
 
 __host__ __device__ inline int tmem_cols_for(int n) {
   int c = 32;
@@ -189,6 +195,19 @@ __device__ __forceinline__ void cluster_arrive_relaxed() {
 }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 
+// Non-blocking test of the completion of phase `parity` of an mbarrier.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(ptx::smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bulk copy of `bytes` from this CTA's shared memory to another CTA's shared
 // memory of the cluster; completion is counted in bytes on the destination's mbarrier.
 __device__ __forceinline__ void bulk_copy_to_rank(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
@@ -209,7 +228,8 @@ constexpr int kGemmThreads = 64 + kEpiThreads;
 
 // (Two CTAs fit an SM by registers, so a grid a little larger than the SM
 // count still runs in one wave.)
-template <int MODE>
+// F8: the weights are FP8 E4M3 codes (GU and DOWN of an FP8 MLP), a.wt8 set.
+template <int MODE, bool F8>
 __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   constexpr int kMaxOwn = 160;   // tokens one rank reduces and finishes
@@ -224,10 +244,11 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
   const int n_mma = min(a.tt, n_rows - t0);
   const int T = min(a.T - t0, n_mma);
   const int cs = gridDim.x;
-  const bool f8 = (MODE == GM_GU || MODE == GM_DOWN) && a.wt8 != nullptr;
+  constexpr bool f8 = F8 && (MODE == GM_GU || MODE == GM_DOWN);
   const GemmSmem L = gemm_smem_layout(a.stages, n_mma, cs, T, MODE != GM_GU, f8);
   // every CTA of a cluster sees the same values, so a refusal is uniform across it
-  if (dynamic_smem_size() < (uint32_t)L.total || a.kslice < 64 || (a.kslice & 63) || a.stages < 1 || n_mma > 256 ||
+  if (dynamic_smem_size() < (uint32_t)L.total || (a.wt8 != nullptr) != f8 || a.kslice < 64 || (a.kslice & 63) ||
+      a.stages < 1 || n_mma > 256 ||
       n_mma < 16 || (n_mma & 15) || (n_rows & 15) || T < 1 || T > n_mma || cs > 16 || (T + cs - 1) / cs > kMaxOwn) {
     if (threadIdx.x == 0) atomicOr(a.status, RTV_DEV_BOUNDS);
     return;
@@ -244,8 +265,13 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
   const int n_own = max(0, min(T, t_own0 + per) - t_own0);
   float* part = (float*)(base + L.part_off);           // [n_mma][128] this CTA's partial sums
   float* recv = (float*)(base + L.recv_off);           // [cs][per][128] partials of the tokens I own
-  uint64_t* full = (uint64_t*)(base + L.bar_off);      // weight + activation boxes landed
-  uint64_t* empty = full + NS;                         // the stage's MMAs completed
+  // bf16: the stage's weight and activation boxes both land on wfull; FP8:
+  // the weight box lands on wfull (the converters wait for it alone) and the
+  // activation box on afull
+  uint64_t* wfull = (uint64_t*)(base + L.bar_off);
+  uint64_t* afull = wfull + NS;
+  uint64_t* abar = f8 ? afull : wfull;                 // where the activation boxes land
+  uint64_t* empty = afull + NS;                        // the stage's MMAs completed
   uint64_t* conv = empty + NS;                         // FP8: the stage's weights widened to bf16
   uint64_t* done = conv + NS;                          // all MMAs completed
   uint64_t* rbar = done + 1;                           // all partials of my tokens landed
@@ -264,7 +290,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
-      ptx::mbar_init(&full[i], 2);
+      ptx::mbar_init(&wfull[i], f8 ? 1 : 2);
+      ptx::mbar_init(&afull[i], 1);
       ptx::mbar_init(&empty[i], 1);
       ptx::mbar_init(&conv[i], kEpiWarps);
     }
@@ -284,9 +311,9 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
     if (lane == 0) {
       pol = ptx::policy_evict_first();
       for (int b = 0; b < first; ++b) {
-        ptx::mbar_expect_tx(&full[b], wbox_bytes);
-        if (f8) ptx::bulk_load_hint(f8s + b * 8192, wsrc8 + (size_t)b * 8192, 8192u, &full[b], pol);
-        else ptx::bulk_load_hint(base + b * L.stage_bytes, wsrc + (size_t)b * 8192, 16384u, &full[b], pol);
+        ptx::mbar_expect_tx(&wfull[b], wbox_bytes);
+        if (f8) ptx::bulk_load_hint(f8s + b * 8192, wsrc8 + (size_t)b * 8192, 8192u, &wfull[b], pol);
+        else ptx::bulk_load_hint(base + b * L.stage_bytes, wsrc + (size_t)b * 8192, 16384u, &wfull[b], pol);
       }
       if (trace) trace[TR_W_ISSUED] = ptx::globaltimer();
     } else if (lane == 2 && a.pf && blockIdx.y == 0) {
@@ -315,21 +342,24 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
 
   // After a bounded wait gives up, a role stops issuing copies and MMAs (so no
   // barrier ever sees an extra arrival), records the timeout, and still
-  // reaches every cluster barrier.
+  // reaches every cluster barrier; what it had issued is drained before exit.
+  int n_issued = 0;   // lane 0: weight boxes, lane 1: activation boxes requested
   if (warp == 0) {
     // ---- producers: lane 0 streams the remaining weight boxes as stages free
     // up; lane 1 the activation boxes once the previous kernel is done (two
     // issuing threads keep more copies in flight per SM) ----
     if (lane == 0) {
+      n_issued = first;
       for (int b = first; b < nbox; ++b) {
         const int s = b % NS, u = b / NS;
         if (!ptx::mbar_wait(&empty[s], (u - 1) & 1, a.timeout_ns)) {
           atomicOr(a.status, RTV_DEV_TIMEOUT);
           break;
         }
-        ptx::mbar_expect_tx(&full[s], wbox_bytes);
-        if (f8) ptx::bulk_load_hint(f8s + s * 8192, wsrc8 + (size_t)b * 8192, 8192u, &full[s], pol);
-        else ptx::bulk_load_hint(base + s * L.stage_bytes, wsrc + (size_t)b * 8192, 16384u, &full[s], pol);
+        ptx::mbar_expect_tx(&wfull[s], wbox_bytes);
+        if (f8) ptx::bulk_load_hint(f8s + s * 8192, wsrc8 + (size_t)b * 8192, 8192u, &wfull[s], pol);
+        else ptx::bulk_load_hint(base + s * L.stage_bytes, wsrc + (size_t)b * 8192, 16384u, &wfull[s], pol);
+        n_issued = b + 1;
       }
     } else if (lane == 1) {
       ptx::pdl_wait();
@@ -340,18 +370,19 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
           atomicOr(a.status, RTV_DEV_TIMEOUT);
           break;
         }
-        ptx::mbar_expect_tx(&full[s], act_box_bytes);
-        ptx::bulk_load(base + s * L.stage_bytes + 16384, asrc + (size_t)b * n_rows * 64, act_box_bytes, &full[s]);
+        ptx::mbar_expect_tx(&abar[s], act_box_bytes);
+        ptx::bulk_load(base + s * L.stage_bytes + 16384, asrc + (size_t)b * n_rows * 64, act_box_bytes, &abar[s]);
+        n_issued = b + 1;
       }
     }
   } else if (warp == 1) {
     // ---- MMA issue: one thread ----
     if (lane == 0) {
       const uint32_t idesc = ptx::idesc_bf16_f32(128, n_mma);
-      uint64_t* ready = f8 ? conv : full;   // FP8: the converters have seen the stage land and widened it
+      uint64_t* wready = f8 ? conv : wfull;   // FP8: the converters have seen the stage land and widened it
       for (int b = 0; b < nbox; ++b) {
         const int s = b % NS, u = b / NS;
-        if (!ptx::mbar_wait(&ready[s], u & 1, a.timeout_ns)) {
+        if (!ptx::mbar_wait(&wready[s], u & 1, a.timeout_ns) || (f8 && !ptx::mbar_wait(&afull[s], u & 1, a.timeout_ns))) {
           atomicOr(a.status, RTV_DEV_TIMEOUT);
           break;
         }
@@ -368,12 +399,45 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
         }
         ptx::umma_commit(&empty[s]);
       }
+      // (also after a break: `done` then completes once the MMAs issued so far have)
       ptx::umma_commit(done);
       if (trace) trace[TR_MMA_ISSUED] = ptx::globaltimer();
     }
   } else {
     // ---- epilogue warps 2..9 ----
     const int tid = threadIdx.x - 64;
+    // FP8 weights: per-row scales of this lane's features, and the widening
+    // of every stage's E4M3 box into the bf16 operand tile.  The first
+    // ring-full does not depend on the previous kernel, so it is widened
+    // before waiting on that kernel; later boxes as their stages come round.
+    const int f0 = 2 * lane;
+    float2 ws1 = make_float2(1.f, 1.f), ws2 = make_float2(1.f, 1.f);
+    bool conv_ok = true;
+    auto widen = [&](int b) {
+      const int s = b % NS, u = b / NS;
+      if (!conv_ok) return;
+      // (a warp-uniform decision: the __syncwarp below needs every lane)
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&wfull[s], u & 1, a.timeout_ns))) {
+        if (lane == 0) atomicOr(a.status, RTV_DEV_TIMEOUT);
+        conv_ok = false;   // the MMA warp then times out on conv[s] and stops issuing
+        return;
+      }
+      const uint8_t* src = f8s + s * 8192;          // [128 rows][64 codes]
+      uint8_t* dst = base + s * L.stage_bytes;       // [128 rows][64 bf16], 128-byte swizzle
+      for (int q = tid; q < 1024; q += kEpiThreads) {
+        const int r = q >> 3, c = q & 7;             // 8 codes -> one 16-byte chunk
+        const uint2 codes = *reinterpret_cast<const uint2*>(src + r * 64 + c * 8);
+        *reinterpret_cast<uint4*>(dst + r * 128 + ((c ^ (r & 7)) << 4)) = e4m3x8_to_bf16x8(codes);
+      }
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&conv[s]);
+    };
+    if (f8) {
+      ws1 = *reinterpret_cast<const float2*>(a.wscale + nt * 128 + f0);
+      ws2 = *reinterpret_cast<const float2*>(a.wscale + nt * 128 + 64 + f0);
+      for (int b = 0; b < first; ++b) widen(b);
+    }
     ptx::pdl_wait();   // this role reads and writes what earlier kernels produced
     if (tid == 0 && cs > 1) ptx::mbar_expect_tx(rbar, (uint32_t)(cs * n_own * 512));
     // Everything the epilogue reads from global memory depends only on earlier
@@ -400,7 +464,6 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
       }
     }
     // gains of the next norm for this lane's features (O, DOWN)
-    const int f0 = 2 * lane;
     const int n1 = nt * 128 + f0, n2 = n1 + 64;
     float2 gn1 = make_float2(0.f, 0.f), gn2 = make_float2(0.f, 0.f);
     if ((MODE == GM_O || MODE == GM_DOWN) && a.g_next) {
@@ -412,31 +475,12 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
       for (int j2 = 0; j2 < n_wt; ++j2) sst += a.ssp[(size_t)(t0 + t_own0 + tid) * n_wt + j2];
       rs_s[tid] = rsqrtf(sst / (float)a.w + a.eps);
     }
-    // FP8 weights: per-row scales of this lane's features, and the widening
-    // of every stage's E4M3 box into the bf16 operand tile while the MMAs run
-    float2 ws1 = make_float2(1.f, 1.f), ws2 = make_float2(1.f, 1.f);
-    if (f8) {
-      ws1 = *reinterpret_cast<const float2*>(a.wscale + nt * 128 + f0);
-      ws2 = *reinterpret_cast<const float2*>(a.wscale + nt * 128 + 64 + f0);
-      for (int b = 0; b < nbox; ++b) {
-        const int s = b % NS, u = b / NS;
-        if (!ptx::mbar_wait(&full[s], u & 1, a.timeout_ns)) {
-          atomicOr(a.status, RTV_DEV_TIMEOUT);
-          break;
-        }
-        const uint8_t* src = f8s + s * 8192;          // [128 rows][64 codes]
-        uint8_t* dst = base + s * L.stage_bytes;       // [128 rows][64 bf16], 128-byte swizzle
-        for (int q = tid; q < 1024; q += kEpiThreads) {
-          const int r = q >> 3, c = q & 7;             // 8 codes -> one 16-byte chunk
-          const uint2 codes = *reinterpret_cast<const uint2*>(src + r * 64 + c * 8);
-          *reinterpret_cast<uint4*>(dst + r * 128 + ((c ^ (r & 7)) << 4)) = e4m3x8_to_bf16x8(codes);
-        }
-        ptx::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&conv[s]);
-      }
+    if (f8)
+      for (int b = first; b < nbox; ++b) widen(b);
+    if (!ptx::mbar_wait(done, 0, a.timeout_ns)) {
+      atomicOr(a.status, RTV_DEV_TIMEOUT);
+      ptx::mbar_wait(done, 0, kDrainNs);   // the MMAs issued so far complete on their own
     }
-    if (!ptx::mbar_wait(done, 0, a.timeout_ns)) atomicOr(a.status, RTV_DEV_TIMEOUT);
     ptx::tc_fence_after();
     if (trace && tid == 0) trace[TR_DONE] = ptx::globaltimer();
     // accumulator -> this CTA's partial tile [token][feature]; the two warps
@@ -473,7 +517,12 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
     ptx::cp_async_wait_all();
     asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
     if (trace && tid == 0) trace[TR_PREFETCHED] = ptx::globaltimer();
-    if (cs > 1 && !ptx::mbar_wait(rbar, 0, a.timeout_ns)) atomicOr(a.status, RTV_DEV_TIMEOUT);
+    // (every rank sends its copies unconditionally, so a wait that runs out
+    // still drains them before this CTA lets anyone leave)
+    if (cs > 1 && !ptx::mbar_wait(rbar, 0, a.timeout_ns)) {
+      atomicOr(a.status, RTV_DEV_TIMEOUT);
+      ptx::mbar_wait(rbar, 0, kDrainNs);
+    }
     if (trace && tid == 0) trace[TR_RECV] = ptx::globaltimer();
     // My incoming copies are complete (seen on rbar), so the copies that read
     // the senders' shared memory are done too; the arrive needs no ordering.
@@ -606,9 +655,19 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, ncols);
   }
-  // never leave with a copy still landing in this CTA's shared memory
-  if (warp == 0 && lane == 0) {
-    for (int s2 = 0; s2 < first; ++s2) ptx::mbar_wait(&full[s2], ((nbox - 1 - s2) / NS) & 1, a.timeout_ns);
+  // Never leave with a copy still landing in this CTA's shared memory: each
+  // producer checks the last box it requested on every stage (copies land in
+  // order of request per stage, so that is the newest phase of the stage).
+  // Unless a wait ran out, every one was consumed by a completed MMA and the
+  // check is a single non-blocking test; otherwise it waits for the copy.
+  if (warp == 0 && lane < 2) {
+    uint64_t* landed = lane == 0 ? wfull : abar;
+    for (int s2 = 0; s2 < NS && s2 < n_issued; ++s2) {
+      const int b_last = s2 + NS * ((n_issued - 1 - s2) / NS);
+      const uint32_t par = (uint32_t)(b_last / NS) & 1;
+      if (!mbar_test(&landed[s2], par) && !ptx::mbar_wait(&landed[s2], par, kDrainNs))
+        atomicOr(a.status, RTV_DEV_TIMEOUT);
+    }
   }
 }
 
@@ -930,6 +989,7 @@ template <int D>
 __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const AttnTcArgs a) {
   extern __shared__ uint8_t sm_atc[];
   __shared__ float red_m[2][128], red_l[2][128];   // per-row partial max / sum of the two column halves
+  __shared__ int s_timeout;                        // a wait of this CTA ran out: drain before leaving
   constexpr int QB = 128 * D * 2, KB = 64 * D * 2, VB = D * 64 * 2, PB = 128 * 128;
   // Tensor memory: S in columns [0, 64), then O in columns [0, D) -- the PV
   // MMA is issued only after every thread has read S.  At most D <= 256
@@ -967,6 +1027,7 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const AttnTcArgs a) {
           : nullptr;
   if (trace && tid == 0) trace[0] = ptx::globaltimer();
   if (tid == 0) {
+    s_timeout = 0;
     for (int i = 0; i < 4; ++i) ptx::mbar_init(&bars[i], 1);
     ptx::fence_mbar_init();
   }
@@ -999,7 +1060,10 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const AttnTcArgs a) {
     ptx::mbar_expect_tx(&bars[1], (uint32_t)QB);
     const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(a.qt + (size_t)(g * HP + hp) * 128 * D);
     for (int c = 0; c < QB; c += 16384) ptx::bulk_load(Qs + c, qsrc + c, 16384u, &bars[1]);
+  }
+  if (tid == 0) {
     ok = ptx::mbar_wait(&bars[1], 0, a.timeout_ns) && ptx::mbar_wait(&bars[0], 0, a.timeout_ns);
+    if (!ok) atomicOr(&s_timeout, 1);
     if (ok) {
       if (trace) trace[2] = ptx::globaltimer();
       ptx::tc_fence_after();
@@ -1025,7 +1089,10 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const AttnTcArgs a) {
   const int n_keys = suffix_tile ? (a.mask_mode == kMaskPrefixOnly ? 0 : a.S) : min(64, a.P - 64 * rank);
   // the Pi0 block mask hides the action tokens of the suffix from the state token (row s == 0)
   const int n_vis = (a.mask_mode == RTV_MASK_PI0_BLOCK && suffix_tile && s == 0) ? 1 : n_keys;
-  if (!ptx::mbar_wait(&bars[2], 0, a.timeout_ns)) atomicOr(a.status, RTV_DEV_TIMEOUT);
+  if (!ptx::mbar_wait(&bars[2], 0, a.timeout_ns)) {
+    atomicOr(a.status, RTV_DEV_TIMEOUT);
+    atomicOr(&s_timeout, 1);
+  }
   ptx::tc_fence_after();
   if (trace && tid == 0) trace[9] = ptx::globaltimer();
   float x[32];
@@ -1078,7 +1145,10 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const AttnTcArgs a) {
     ptx::umma_commit(&bars[3]);
   }
   __syncwarp();
-  if (!ptx::mbar_wait(&bars[3], 0, a.timeout_ns)) atomicOr(a.status, RTV_DEV_TIMEOUT);
+  if (!ptx::mbar_wait(&bars[3], 0, a.timeout_ns)) {
+    atomicOr(a.status, RTV_DEV_TIMEOUT);
+    atomicOr(&s_timeout, 1);
+  }
   ptx::tc_fence_after();
   if (trace && tid == 0) trace[4] = ptx::globaltimer();
   // unnormalised O rows -> the Q tile's space (free since S was computed),
@@ -1181,15 +1251,22 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const AttnTcArgs a) {
     }
   }
   if (trace && tid == 0) trace[8] = ptx::globaltimer();
+  // Never leave, or free the tensor memory, with a copy or an MMA of this CTA
+  // still in flight (they complete on their own; after a timeout above this
+  // drains them).  Every copy was requested; the MMAs only when `ok`.
+  ptx::tc_fence_before();
   __syncthreads();
+  if (s_timeout) {   // (uniform: read after the barrier)
+    if (tid == 0) {
+      bool drained = ptx::mbar_wait(&bars[0], 0, kDrainNs) && ptx::mbar_wait(&bars[1], 0, kDrainNs);
+      if (ok) drained = drained && ptx::mbar_wait(&bars[2], 0, kDrainNs) && ptx::mbar_wait(&bars[3], 0, kDrainNs);
+      if (!drained) atomicOr(a.status, RTV_DEV_TIMEOUT);
+    }
+    __syncthreads();
+  }
   if (warp == 0) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, TCOLS);
-  }
-  // never leave with a copy still landing in this CTA's shared memory
-  if (tid == 0 && !ok) {
-    ptx::mbar_wait(&bars[0], 0, a.timeout_ns);
-    ptx::mbar_wait(&bars[1], 0, a.timeout_ns);
   }
 }
 
@@ -1566,7 +1643,7 @@ GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T, bool with
 template <int MODE>
 cudaError_t launch_gemm(const GemmArgs& a, const GemmPlan& pl, cudaStream_t st,
                         unsigned long long pf_cap = ~0ull) {
-  auto kern = gemm_tc_kernel<MODE>;
+  auto kern = a.wt8 ? gemm_tc_kernel<MODE, true> : gemm_tc_kernel<MODE, false>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.cs, pl.n_tt, pl.n_tiles);
   cfg.blockDim = dim3(kGemmThreads, 1, 1);
@@ -1602,8 +1679,11 @@ cudaError_t configure_dyn_smem(K kern) {
 // Kernel attributes are set once, outside any stream capture.
 template <int MODE>
 cudaError_t configure_gemm() {
-  cudaError_t e = configure_dyn_smem(gemm_tc_kernel<MODE>);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(gemm_tc_kernel<MODE>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaError_t e = cudaSuccess;
+  for (auto kern : {gemm_tc_kernel<MODE, false>, gemm_tc_kernel<MODE, true>}) {
+    if (e == cudaSuccess) e = configure_dyn_smem(kern);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  }
   return e;
 }
 
@@ -1751,7 +1831,7 @@ rtv_status fast_create(rtv_ctx* ctx) {
       cfg.attrs = &at;
       cfg.numAttrs = 1;
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<GM_DOWN>, &cfg) != cudaSuccess) n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<GM_DOWN, false>, &cfg) != cudaSuccess) n = 0;
       cudaGetLastError();
       (big ? fp->gemm_fit_large : fp->gemm_fit_small)[cs] = n;
     }

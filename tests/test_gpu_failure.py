@@ -4,12 +4,13 @@
   output head records RTV_DEV_NUMERIC, rtv_device_status reports
   RTV_ERR_NUMERIC, and the next clean call on the same context is correct
   (no state of the context keeps the NaN).
-* A device-side wait that runs out: the resident kernel given a wait limit of
-  two microseconds cannot pass its first grid barrier in time.  Every CTA
-  stops issuing work, waits for the copies and MMAs it already issued, frees
-  its tensor memory and returns; the status word reports RTV_DEV_TIMEOUT and
-  the context stays usable (a second call reports the same, no CUDA error),
-  and a context with the default limit then computes the chunk correctly.
+* A device-side wait that runs out: the layered kernels given a wait limit of
+  one nanosecond, and the resident kernel given two microseconds (it cannot
+  pass its first grid barrier in time).  Every CTA stops issuing work, waits
+  for the copies and MMAs it already issued, frees its tensor memory and
+  returns; the status word reports RTV_DEV_TIMEOUT and the context stays
+  usable (a second call reports the same, no CUDA error), and a context with
+  the default limit then computes the chunk correctly.
 """
 
 import numpy as np
@@ -44,13 +45,17 @@ def test_nan_input_is_reported_and_the_next_call_is_clean(cuda_ok, monkeypatch, 
     ex.close()
 
 
-def test_wait_that_runs_out_is_reported_and_the_context_stays_usable(cuda_ok, monkeypatch):
-    monkeypatch.setenv("RTV_PATH", "resident")
+# Wait limits that run out on every launch: the layered kernels' first wait on
+# a copy (a weight box is ~1 us away when the MMA thread first looks) at 1 ns;
+# the resident kernel's first grid barrier at 2 us.
+@pytest.mark.parametrize("path,limit_ns", [("layered", 1), ("resident", 2000)])
+def test_wait_that_runs_out_is_reported_and_the_context_stays_usable(cuda_ok, monkeypatch, path, limit_ns):
+    monkeypatch.setenv("RTV_PATH", path)
     cfg = get_config("pi0-bf16", n_layers=1, prefix_len=64)
     weights = make_weights(cfg)
     kv = np.ascontiguousarray(f32_to_bf16_bits(make_prefix_kv(cfg)))
     noise, state = make_noise(cfg), make_state(cfg)
-    ex = ActionExpert(cfg, barrier_timeout_ns=2000)
+    ex = ActionExpert(cfg, barrier_timeout_ns=limit_ns)
     ex.load(weights)
     ex.set_prefix_kv(kv)
     for _ in range(2):
