@@ -25,6 +25,8 @@ region.  `cpu_baseline` times the CPU oracle on a bounded sample.
 from __future__ import annotations
 
 import argparse
+import glob
+import hashlib
 import json
 import os
 import statistics
@@ -88,6 +90,24 @@ def algorithmic_bytes_per_step(cfg, batch=1):
         proj += 2 * w * w * elt
     kv = 2 * batch * cfg.prefix_len * cfg.kv_dim * elt
     return cfg.n_layers * (layer + kv) + proj
+
+
+# DRAM bytes (read + written) of one pi0-bf16 chunk (18 layers, P = 816, batch 1), summed by ncu over the 911
+# launches of a chunk with the L2 carried between kernels (profiles/dram_traffic_pi0-bf16_full_depth.md).  The
+# figure holds for the kernel sources it was taken on, identified by their SHA-256; after any change to them the
+# bench reports null until the capture is taken again.
+TRAFFIC_PI0_BF16 = {"bytes_per_chunk": 6436052736,
+                    "kernel_sources_sha256": "c7aa151cc32c9f6ae92ed95a6cdaf610d4242bbfcf549af84e5e766163cc7763"}
+
+
+def kernel_sources_sha256():
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "flow_matching_action_dm0_b200", "csrc", "*"))):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(os.path.basename(f).encode())
+            with open(f, "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()
 
 
 def load_peaks():
@@ -456,6 +476,15 @@ def run_ours(args, info):
     bytes_chunk = bytes_step * n
     achieved = bytes_chunk / (ms * 1e-3) / 1e9
     peak = float(peaks["hbm_gbs"])
+    traffic, traffic_note = None, "DRAM bytes were captured for pi0-bf16 at full depth only"
+    if args.workload == "pi0-bf16" and args.layers <= 0 and n == 10 and cfg.batch == 1:
+        if kernel_sources_sha256() == TRAFFIC_PI0_BF16["kernel_sources_sha256"]:
+            traffic = TRAFFIC_PI0_BF16["bytes_per_chunk"]
+            traffic_note = ("ncu dram__bytes_read.sum + dram__bytes_write.sum over the 911 launches of one chunk, "
+                            "L2 carried between kernels; bytes per chunk (traffic / algorithmic = "
+                            f"{traffic / bytes_chunk:.3f})")
+        else:
+            traffic_note = "the kernel sources changed since the DRAM capture: not yet taken again"
     line = {
         "metric": METRIC,
         "value": ms * 1000.0,
@@ -478,12 +507,8 @@ def run_ours(args, info):
         "roofline": {"bound": "hbm", "kernel": "whole denoise graph (all kernels of one chunk)",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_kind": f"{peak_kind} hbm_gbs", "algorithmic_bytes_per_launch": bytes_chunk,
-                     "traffic": None,
-                     "traffic_note": "DRAM bytes not captured at full depth (multi-pass ncu at 18 layers is "
-                                     "avoided); an ncu capture of a 6-layer expert with the cache carried "
-                                     "between kernels read 26.6 MB per layer-step against 35.4 MB algorithmic "
-                                     "(no weight byte read twice; the rest is cross-step L2 reuse that 6 layers "
-                                     "allow and 18 do not)"},
+                     "traffic": traffic,
+                     "traffic_note": traffic_note},
         "e2e": {"value": e2e_ms * 1000.0, "unit": "us",
                 "h2d_bytes_per_step": int(noise.nbytes + state.nbytes), "d2h_bytes_per_step": int(noise.nbytes)},
         "latency": latency,
