@@ -986,16 +986,18 @@ struct AttnTcArgs {
 __host__ __device__ inline int attn_tc_smem_bytes(int D) { return 128 * D * 2 + 2 * 64 * D * 2 + 128 * 128 + 64 + 1024; }
 
 template <int D>
-__global__ void __launch_bounds__(256, 1) attn_tc_kernel(const AttnTcArgs a) {
+__global__ void __launch_bounds__(256, 2) attn_tc_kernel(const AttnTcArgs a) {
   extern __shared__ uint8_t sm_atc[];
   __shared__ float red_m[2][128], red_l[2][128];   // per-row partial max / sum of the two column halves
   __shared__ int s_timeout;                        // a wait of this CTA ran out: drain before leaving
   constexpr int QB = 128 * D * 2, KB = 64 * D * 2, VB = D * 64 * 2, PB = 128 * 128;
   // Tensor memory: S in columns [0, 64), then O in columns [0, D) -- the PV
   // MMA is issued only after every thread has read S.  At most D <= 256
-  // columns, so this CTA and any GEMM CTA sharing its SM (at most 256
-  // columns each, and shared memory admits no third) never exceed the 512
-  // columns: no allocation ever waits on a CTA of a later kernel.
+  // columns, so two CTAs sharing an SM (two attention CTAs, which a grid
+  // larger than the SM count places together, or one beside a GEMM CTA of
+  // at most 256 columns; shared memory admits no third) never exceed the 512
+  // columns.  An allocation can only wait for a CTA of an earlier kernel,
+  // which never waits on a later one.
   constexpr uint32_t TCOLS = D;
   constexpr int CPR = D / 8;
   const int nch = gridDim.x;
@@ -1186,26 +1188,32 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const AttnTcArgs a) {
   // release / acquire at cluster scope: every rank's partials are visible
   ptx::cluster_sync();
   if (trace && tid == 0) trace[6] = trace[7] = ptx::globaltimer();
+  constexpr int kRB = 1;   // rows per warp step (one row's 16 loads in flight keeps two CTAs per SM)
   // combine: the pair's 2*S valid rows are split evenly over the ranks; a warp
-  // takes two of its rank's rows at a time and issues every load of both
+  // takes one of its rank's rows at a time and issues every load of it
   // before reducing (ranks summed in order)
   const int nvalid = 2 * a.S;
   const int rpc = (nvalid + nch - 1) / nch;
   const int v0 = rank * rpc, v1 = min(nvalid, v0 + rpc);
-  for (int vb = v0 + warp; vb < v1; vb += 16) {
-    int rows[2];
-    bool has[2];
+  for (int vb = v0 + warp; vb < v1; vb += 8 * kRB) {
+    int rows[kRB];
+    bool has[kRB];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < kRB; ++u) {
       const int vi = vb + 8 * u;
       has[u] = vi < v1;
       const int hs = has[u] ? vi / a.S : 0;
       rows[u] = has[u] ? hs * 64 + (vi - hs * a.S) : 0;
     }
-    float mq[2] = {-INFINITY, -INFINITY}, lq[2] = {0.f, 0.f};
-    uint4 v[2][16];
+    float mq[kRB], lq[kRB];
+    uint4 v[kRB][16];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < kRB; ++u) {
+      mq[u] = -INFINITY;
+      lq[u] = 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kRB; ++u) {
       if (has[u] && lane < nch) {
         const float2 ml =
             __ldcg(reinterpret_cast<const float2*>(a.part_ml + ((part_base + lane) * 128 + rows[u]) * 2));
@@ -1219,7 +1227,7 @@ __global__ void __launch_bounds__(256, 1) attn_tc_kernel(const AttnTcArgs a) {
     }
     if (trace && tid == 0 && vb == v0) trace[13] = ptx::globaltimer();
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < kRB; ++u) {
       if (!has[u]) continue;   // uniform across the warp
       const float m_all = warp_max(mq[u]);
       const float wq = (lane < nch && mq[u] != -INFINITY) ? exp2f(mq[u] - m_all) : 0.f;
