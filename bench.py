@@ -537,13 +537,19 @@ def run_ours(args, info):
 
 def draft_bytes(dcfg) -> int:
     """Algorithmic bytes of one draft forward: the block's and head's weights,
-    the queries, the image features read, and their keys/values written and
-    read back once."""
+    the queries' residual rows, the image features read, and their keys/values
+    written and read back once.  On the tensor-core path (bf16) the action
+    queries' q/k/v depend on the weights only and are computed once per graph:
+    a forward reads their tiles instead of the q projection's weights."""
     e = 2 if dcfg.dtype == "bf16" else 4
     w = dcfg.width
     kv = dcfg.n_vis * 2 * dcfg.kv_dim * e
-    return (dcfg.block_params() - 2 * w) * e + 2 * w * 4 + dcfg.action_dim * (w * e + 4) + \
+    total = (dcfg.block_params() - 2 * w) * e + 2 * w * 4 + dcfg.action_dim * (w * e + 4) + \
         dcfg.n_queries * w * 4 + dcfg.n_vis * w * e + 2 * kv
+    if dcfg.dtype == "bf16":
+        folded_tiles = (dcfg.n_q_heads // 2) * 128 * dcfg.head_dim * 2 + 2 * dcfg.n_kv_heads * 64 * dcfg.head_dim * 2
+        total += folded_tiles - w * dcfg.q_dim * e
+    return total
 
 
 def measure_round(ex, cfg, noise, state, stream, dev, K):

@@ -168,9 +168,10 @@ __global__ void vis_kv_store_kernel(const float* __restrict__ kv, const float* _
 }
 
 // The draft forward for (V, B), enqueued on st (captured into a graph).
+// fold: the query rows' layer-0 tiles and residual, computed at graph build.
 template <typename WT>
 rtv_status enqueue_forward(rtv_draft* d, int V, int B, const float* cs_v, const float* sn_v, const float* cs_q,
-                           const float* sn_q, cudaStream_t st) {
+                           const float* sn_q, const FoldedQueries* fold, cudaStream_t st) {
   rtv_ctx* c = d->blk;
   const rtv_expert_config& k = c->cfg;
   const int w = k.width, H = d->cfg.n_queries, A = d->cfg.action_dim;
@@ -178,8 +179,12 @@ rtv_status enqueue_forward(rtv_draft* d, int V, int B, const float* cs_v, const 
   const int Tv = B * V, Tq = B * H;
   if (c->use_fast) {
     DTRY(fast_block_prefix(c, (const __nv_bfloat16*)d->vis_in, V, B, d->vis_hb, d->vis_ssp, cs_v, sn_v, st));
-    DTRY(fast_block_embed(c, d->queries, H, B, st));
-    DTRY(fast_layers(c, B, V, 1, cs_q, sn_q, st));
+    if (fold) {
+      DTRY(fast_layers(c, B, V, 1, cs_q, sn_q, st, nullptr, fold));
+    } else {
+      DTRY(fast_block_embed(c, d->queries, H, B, st));
+      DTRY(fast_layers(c, B, V, 1, cs_q, sn_q, st));
+    }
   } else {
     const LayerW& L = c->W.layers[0];
     const float* xf = (const float*)d->vis_in;
@@ -219,12 +224,34 @@ rtv_status build_graph(rtv_draft* d, int V, int B, GraphEntry& ge) {
   launch_rope_table(tabs[0], tabs[1], V, D, 0, k.rope_theta, st);
   launch_rope_table(tabs[2], tabs[3], H, D, V, k.rope_theta, st);
   DCK(cudaGetLastError());
+  // The action queries are weights: the first norm of their rows, their q, k
+  // and v (RoPE at V..V+H-1) and the residual the O projection adds to depend
+  // on the weights and V only, so they are computed here, once per graph, and
+  // the forward starts the query rows at the attention.
+  FoldedQueries fold;
+  const bool folding = c->use_fast && fast_tc_attention(c, V);
+  if (folding) {
+    size_t bytes[4];
+    folded_sizes(c, B, bytes);
+    void* p[4] = {nullptr, nullptr, nullptr, nullptr};
+    for (int i = 0; i < 4; ++i) {
+      DCK(cudaMalloc(&p[i], bytes[i]));
+      ge.owned.push_back(p[i]);
+    }
+    fold.qt = (__nv_bfloat16*)p[0];
+    fold.kts = (__nv_bfloat16*)p[1];
+    fold.vts = (__nv_bfloat16*)p[2];
+    fold.h0 = (float*)p[3];
+    const rtv_status s = fast_block_fold(c, d->queries, H, B, V, tabs[2], tabs[3], fold, st);
+    if (s != RTV_OK) return dfail(d, s, c->last_error);
+  }
   DCK(cudaStreamSynchronize(st));
   c->last_error.clear();
   DCK(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
+  const FoldedQueries* fp = folding ? &fold : nullptr;
   const rtv_status fs = k.dtype == RTV_F32
-                            ? enqueue_forward<float>(d, V, B, tabs[0], tabs[1], tabs[2], tabs[3], st)
-                            : enqueue_forward<__nv_bfloat16>(d, V, B, tabs[0], tabs[1], tabs[2], tabs[3], st);
+                            ? enqueue_forward<float>(d, V, B, tabs[0], tabs[1], tabs[2], tabs[3], fp, st)
+                            : enqueue_forward<__nv_bfloat16>(d, V, B, tabs[0], tabs[1], tabs[2], tabs[3], fp, st);
   cudaGraph_t g = nullptr;
   const cudaError_t e1 = cudaGetLastError();
   const cudaError_t e2 = cudaStreamEndCapture(st, &g);

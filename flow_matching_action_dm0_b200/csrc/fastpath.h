@@ -18,6 +18,8 @@ rtv_status fast_create(rtv_ctx* ctx);
 // Pack the loaded parameters into the tensor-core layouts.
 rtv_status fast_load(rtv_ctx* ctx, const rtv_tensor* params, int n_params);
 bool fast_supports_prefix(rtv_ctx* ctx, int prefix_len);
+// Whether the tensor-core attention serves a prefix of P keys (else the warp-MMA one).
+bool fast_tc_attention(const rtv_ctx* ctx, int P);
 // Refresh the tensor-core layouts of the cached prefix after ctx->prefix_kv changed.
 rtv_status fast_prefix_update(rtv_ctx* ctx, int batch, int prefix_len, cudaStream_t st);
 // Step boundary over G suffixes: output head (Euler update of ctx->x, or the
@@ -28,10 +30,29 @@ rtv_status fast_prefix_update(rtv_ctx* ctx, int batch, int prefix_len, cudaStrea
 rtv_status fast_step(rtv_ctx* ctx, int G, bool do_head, bool do_embed, float dt, const float* c, int c_stride,
                      int state_stride, bool velocity_only, cudaStream_t st, const float* g0 = nullptr,
                      int g0_stride = 0);
+// Layer 0 of a bare block whose suffix rows are weights, not inputs (the
+// FLASH draft's learnable action queries): their q and suffix K/V tiles and
+// residual rows depend on the weights and the RoPE positions only, so they
+// are computed once (fast_block_fold) and read in place of a QKV projection.
+struct FoldedQueries {
+  __nv_bfloat16* qt = nullptr;    // [G][Hq/2][128][D] tiled q of the head pairs
+  __nv_bfloat16* kts = nullptr;   // [G][Hkv][64][D] tiled suffix keys
+  __nv_bfloat16* vts = nullptr;   // [G][Hkv][D][64] tiled suffix values (transposed)
+  float* h0 = nullptr;            // [G*S][width] residual rows the O projection adds to
+};
 // The expert's layers over G suffixes (residual stream ctx->h); mod set for
-// RTV_TIME_ADARMS.
+// RTV_TIME_ADARMS; fold set: layer 0 reads its query rows' tiles and
+// residual from fold and launches no QKV projection (tensor-core attention only).
 rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, const float* rope_cs,
-                       const float* rope_sn, cudaStream_t st, const ModTables* mod = nullptr);
+                       const float* rope_sn, cudaStream_t st, const ModTables* mod = nullptr,
+                       const FoldedQueries* fold = nullptr);
+// Bytes of the four FoldedQueries buffers for G suffix groups.
+void folded_sizes(const rtv_ctx* ctx, int G, size_t bytes[4]);
+// Bare block: fill f for G suffixes whose residual rows are rows[t % n_src_rows]
+// (RMSNorm, layer 0's QKV projection with RoPE from rope_cs / rope_sn), with a
+// prefix of P keys.  Uses the context's scratch; enqueued on st.
+rtv_status fast_block_fold(rtv_ctx* ctx, const float* rows, int n_src_rows, int G, int P, const float* rope_cs,
+                           const float* rope_sn, const FoldedQueries& f, cudaStream_t st);
 // The first layer's norm input of the residual rows of G suffixes, from ctx->h.
 rtv_status fast_norm_rows(rtv_ctx* ctx, int G, cudaStream_t st);
 // Bare block (ctx->block_only), layer 0: keys and values of n_vis tokens per

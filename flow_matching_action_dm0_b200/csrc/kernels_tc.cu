@@ -96,6 +96,7 @@ struct GemmArgs {
   const uint8_t* pf;          // weights of the next projection, brought into L2 while this one runs
   unsigned long long pf_bytes;
   float* h;                   // fp32 residual stream [T][w] (O, DOWN add into it)
+  const float* h_in;          // O, DOWN: residual rows added to, when not h itself (nullptr: h)
   __nv_bfloat16* hb;          // next norm's input bf16(h * (1 + g_next)), tiled [w/64][n_mma][64] (written by O, DOWN)
   float* ssp;                 // sums of squares of h per 128-feature tile [T][w/128]
   const float* g_next;        // gain of the next RMSNorm, or nullptr when no norm consumer follows
@@ -453,7 +454,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
     if (MODE == GM_O || MODE == GM_DOWN) {
       for (int c = tid; c < n_own * 32; c += kEpiThreads) {
         const int tl = c >> 5, ch = c & 31;
-        ptx::cp_async_16(in_a + (uint32_t)(c * 16), a.h + (size_t)(t0 + t_own0 + tl) * a.w + nt * 128 + ch * 4);
+        ptx::cp_async_16(in_a + (uint32_t)(c * 16),
+                         (a.h_in ? a.h_in : a.h) + (size_t)(t0 + t_own0 + tl) * a.w + nt * 128 + ch * 4);
       }
     } else if (rope) {
       for (int c = tid; c < n_own * 32; c += kEpiThreads) {
@@ -1948,6 +1950,13 @@ void fast_trace_report(rtv_ctx* ctx) {
 
 bool fast_supports_prefix(rtv_ctx*, int) { return true; }
 
+bool fast_tc_attention(const rtv_ctx* ctx, int P) {
+  const FastPath* fp = ctx->fast;
+  const int ntp = (P + 63) / 64;
+  const char* attn_env = getenv("RTV_ATTN");
+  return fp && fp->tc_attn && ntp + 1 <= 16 && ntp <= fp->ntile_max && !(attn_env && strcmp(attn_env, "mma") == 0);
+}
+
 rtv_status fast_prefix_update(rtv_ctx* ctx, int batch, int prefix_len, cudaStream_t st) {
   FastPath* fp = ctx->fast;
   if (!fp || !fp->tc_attn) return RTV_OK;
@@ -2312,8 +2321,14 @@ rtv_status fast_norm_rows(rtv_ctx* ctx, int G, cudaStream_t st) {
   return RTV_OK;
 }
 
-rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, const float* rope_cs,
-                       const float* rope_sn, cudaStream_t st, const ModTables* mod) {
+namespace {
+
+// The layers (see fast_layers); with fold, layer 0 reads its q / suffix K/V
+// tiles and O's residual rows from fold and launches no QKV projection; with
+// qkv0_only, only layer 0's QKV projection is launched.
+rtv_status layers_impl(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, const float* rope_cs,
+                       const float* rope_sn, cudaStream_t st, const ModTables* mod, const FoldedQueries* fold,
+                       bool qkv0_only) {
   FastPath* fp = ctx->fast;
   const rtv_expert_config& k = ctx->cfg;
   const int S = ctx->S, T = G * S, w = k.width, F = k.mlp_dim, D = k.head_dim, Q = ctx->Q, KV = ctx->KV;
@@ -2395,9 +2410,7 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
   // tensor-core attention when the pair layout applies and every key tile has
   // a rank (RTV_ATTN=mma selects the warp-MMA kernel instead)
   const int ntp = (P + 63) / 64;
-  const char* attn_env = getenv("RTV_ATTN");
-  const bool tc_att = fp->tc_attn && ntp + 1 <= 16 && ntp <= fp->ntile_max &&
-                      !(attn_env && strcmp(attn_env, "mma") == 0);
+  const bool tc_att = fast_tc_attention(ctx, P);
   AttnTcArgs atc{};
   if (tc_att) {
     base.qt = fp->qt;
@@ -2435,6 +2448,10 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
   auto tr = [&](int l, int i) -> unsigned long long* {
     return (tracing && l == 0) ? fp->trace + (size_t)i * 512 * kTraceRow : nullptr;
   };
+  if ((fold || qkv0_only) && !tc_att) {
+    ctx->last_error = "folded query rows need the tensor-core attention";
+    return RTV_ERR_UNSUPPORTED;
+  }
 
   // per-layer time modulator rows (RTV_TIME_ADARMS): group strides
   const int L6 = k.n_layers * 6 * w;
@@ -2454,14 +2471,28 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     a.w_tile0 = l * nq / 128;
     a.pf = (const uint8_t*)(fp->w_o + (size_t)l * w * Q);
     a.pf_bytes = (unsigned long long)w * Q * 2;
-    cudaError_t e = launch_gemm<GM_QKV>(a, p_qkv, st, fp->pf_cap);
+    const bool folded = fold && l == 0;
+    cudaError_t e = folded ? cudaSuccess : launch_gemm<GM_QKV>(a, p_qkv, st, fp->pf_cap);
+    if (qkv0_only) {
+      if (e != cudaSuccess) {
+        ctx->last_error = std::string("tensor-core launch: ") + cudaGetErrorString(e);
+        return RTV_ERR_CUDA;
+      }
+      return RTV_OK;
+    }
 
     if (tc_att) {
-      atc.trace = tr(l, 4);
-      atc.pkt = fp->pkt + (size_t)l * ptile_layer;
-      atc.pvt = fp->pvt + (size_t)l * ptile_layer;
+      AttnTcArgs atl = atc;
+      atl.trace = tr(l, 4);
+      atl.pkt = fp->pkt + (size_t)l * ptile_layer;
+      atl.pvt = fp->pvt + (size_t)l * ptile_layer;
+      if (folded) {
+        atl.qt = fold->qt;
+        atl.kts = fold->kts;
+        atl.vts = fold->vts;
+      }
       if (e == cudaSuccess)
-        e = D == 256 ? launch_attn_tc<256>(atc, ntp + 1, G, st) : launch_attn_tc<128>(atc, ntp + 1, G, st);
+        e = D == 256 ? launch_attn_tc<256>(atl, ntp + 1, G, st) : launch_attn_tc<128>(atl, ntp + 1, G, st);
     } else {
       at.trace = tr(l, 4);
       at.pk = (const __nv_bfloat16*)ctx->prefix_kv + (size_t)(2 * l) * kv_layer;
@@ -2478,6 +2509,7 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     a.pf = fp->mlp_f8 ? fp->w_gu8 + (size_t)l * 2 * F * w : (const uint8_t*)(fp->w_gu + (size_t)l * 2 * F * w);
     a.pf_bytes = (unsigned long long)2 * F * w * (fp->mlp_f8 ? 1 : 2);
     a.g_next = Lw.g_mlp;
+    if (folded) a.h_in = fold->h0;
     if (mod) {
       a.gate = ml + 2 * w;
       a.gate_stride = mg * L6;
@@ -2522,6 +2554,42 @@ rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     if (e == cudaSuccess) e = launch_gemm<GM_DOWN>(a, p_dn, st, fp->pf_cap);
     if (e != cudaSuccess) {
       ctx->last_error = std::string("tensor-core launch: ") + cudaGetErrorString(e);
+      return RTV_ERR_CUDA;
+    }
+  }
+  return RTV_OK;
+}
+
+}  // namespace
+
+rtv_status fast_layers(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, const float* rope_cs,
+                       const float* rope_sn, cudaStream_t st, const ModTables* mod, const FoldedQueries* fold) {
+  return layers_impl(ctx, G, P, prefix_batch_stride, rope_cs, rope_sn, st, mod, fold, false);
+}
+
+void folded_sizes(const rtv_ctx* ctx, int G, size_t bytes[4]) {
+  const rtv_expert_config& k = ctx->cfg;
+  const size_t D = k.head_dim;
+  bytes[0] = (size_t)G * (k.n_q_heads / 2) * 128 * D * 2;    // q tiles of the head pairs
+  bytes[1] = (size_t)G * k.n_kv_heads * 64 * D * 2;           // suffix key tiles
+  bytes[2] = bytes[1];                                        // suffix value tiles (transposed)
+  bytes[3] = (size_t)G * ctx->S * k.width * sizeof(float);    // residual rows
+}
+
+rtv_status fast_block_fold(rtv_ctx* ctx, const float* rows, int n_src_rows, int G, int P, const float* rope_cs,
+                           const float* rope_sn, const FoldedQueries& f, cudaStream_t st) {
+  FastPath* fp = ctx->fast;
+  rtv_status s = fast_block_embed(ctx, rows, n_src_rows, G, st);
+  if (s == RTV_OK) s = layers_impl(ctx, G, P, 1, rope_cs, rope_sn, st, nullptr, nullptr, true);
+  if (s != RTV_OK) return s;
+  size_t bytes[4];
+  folded_sizes(ctx, G, bytes);
+  const void* from[4] = {fp->qt, fp->kts, fp->vts, ctx->h};
+  void* to[4] = {f.qt, f.kts, f.vts, f.h0};
+  for (int i = 0; i < 4; ++i) {
+    const cudaError_t e = cudaMemcpyAsync(to[i], from[i], bytes[i], cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) {
+      ctx->last_error = std::string("folding the query rows: ") + cudaGetErrorString(e);
       return RTV_ERR_CUDA;
     }
   }
