@@ -44,7 +44,9 @@ METRIC = "10-step action-chunk latency (us) and achieved HBM GB/s vs 8 TB/s roof
 PREFILL_METRIC = ("prefill + 10-step chunk latency (us): Gemma-2B-class prefill over 816 tokens writing the "
                   "KV cache, then the pi0-bf16 chunk, one CUDA graph")
 DRAFT_METRIC = "FLASH draft forward latency (us): one Gemma-2B-width block + action head over 768 image tokens"
-PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+# Earlier measurements on this machine's B200s, used only when MEASURED_PEAKS.json is absent: a STREAM-style
+# copy, and a cuBLAS bf16 GEMM as a burst and as a seconds-long loop under the power cap.
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
 def parse_args(argv=None):
