@@ -98,8 +98,8 @@ def algorithmic_bytes_per_step(cfg, batch=1):
 # launches of a chunk with the L2 carried between kernels (profiles/dram_traffic_pi0-bf16_full_depth.md).  The
 # figure holds for the kernel sources it was taken on, identified by their SHA-256; after any change to them the
 # bench reports null until the capture is taken again.
-TRAFFIC_PI0_BF16 = {"bytes_per_chunk": 6436052736,
-                    "kernel_sources_sha256": "c7aa151cc32c9f6ae92ed95a6cdaf610d4242bbfcf549af84e5e766163cc7763"}
+TRAFFIC_PI0_BF16 = {"bytes_per_chunk": 6437718272,
+                    "kernel_sources_sha256": "f4692a8b2d6baa7c76d2106bf18e66859fd8cb1281a6d84dc6794d6dcb92d4c2"}
 
 
 def kernel_sources_sha256():
