@@ -1583,7 +1583,9 @@ __global__ void __launch_bounds__(128) norm_input_kernel(const XT* __restrict__ 
 // ===========================================================================
 struct GemmPlan {
   int n_tiles = 0, cs = 1, kslice = 0, stages = 1, smem = 0;
-  int n_tt = 1;   // token tiles (grid z)
+  int n_tt = 1;   // token tiles (grid y)
+  int tt = 0;     // token rows per CTA (0: the caller's)
+  double cost = 0.0;
   bool valid = false;
 };
 
@@ -1623,6 +1625,9 @@ struct FastPath {
   bool trace_armed = false;
   std::vector<void*> allocs;
 };
+
+// Token tiles of a projection over n_mma rows (defined below).
+void token_tiles(int n_mma, int* n_tt, int* tt);
 
 namespace {
 
@@ -1673,6 +1678,7 @@ GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T, bool with
     const double cost = waves * (kFixedBoxes + nbox);
     if (cost < best_cost) {
       best_cost = cost;
+      best.cost = cost;
       best.cs = cs;
       best.kslice = K / cs;
       best.stages = stages;
@@ -1680,6 +1686,36 @@ GemmPlan plan_gemm(const FastPath* fp, int N, int K, int n_mma, int T, bool with
     }
   }
   best.valid = best.kslice >= 64 && best.smem > 0 && best.smem <= kDynSmemMax && (T + best.cs - 1) / best.cs <= 160;
+  return best;
+}
+
+// Plan of a projection of the suffix layers over n_mma token rows (T of them
+// real).  Between 65 and 256 rows the token tiling is chosen with the split:
+// 1-4 tiles, each tile's cluster exchange charged by its rows (about four MMA
+// boxes for every 64 rows beyond the first 64: measured, 160-row tiles made a
+// three-tau verification 13% slower than 64-row ones).
+GemmPlan plan_suffix(const FastPath* fp, int N, int K, int n_mma, int T, bool with_in, bool f8) {
+  int n_tt0 = 1, tt0 = 16;
+  token_tiles(n_mma, &n_tt0, &tt0);
+  if (n_mma <= 64 || n_mma > 256) {
+    GemmPlan p = plan_gemm(fp, N, K, tt0, std::min(T, tt0), with_in, f8, n_tt0);
+    p.tt = tt0;
+    return p;
+  }
+  GemmPlan best;
+  double best_cost = 1e30;
+  for (int n_tt = 1; n_tt <= 4; ++n_tt) {
+    const int tt = round_up((n_mma + n_tt - 1) / n_tt, 16);
+    if ((n_tt - 1) * tt >= n_mma) continue;   // the last tile would be empty
+    GemmPlan p = plan_gemm(fp, N, K, tt, std::min(T, tt), with_in, f8, n_tt);
+    if (!p.valid) continue;
+    const double cost = p.cost + 4.0 * std::max(0, tt - 64) / 64.0;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = p;
+      best.tt = tt;
+    }
+  }
   return best;
 }
 
@@ -1704,6 +1740,7 @@ cudaError_t launch_gemm(const GemmArgs& a, const GemmPlan& pl, cudaStream_t st,
   GemmArgs args = a;
   args.kslice = pl.kslice;
   args.stages = pl.stages;
+  if (pl.tt) args.tt = pl.tt;
   if (args.pf_bytes > pf_cap) args.pf_bytes = pf_cap;
   return cudaLaunchKernelEx(&cfg, kern, args);
 }
@@ -2382,14 +2419,13 @@ rtv_status layers_impl(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
   const rtv_expert_config& k = ctx->cfg;
   const int S = ctx->S, T = G * S, w = k.width, F = k.mlp_dim, D = k.head_dim, Q = ctx->Q, KV = ctx->KV;
   const int n_mma = round_up(T, 16);   // rows of the tiled activation layout
-  int n_tt = 1, tt = 16;               // token tiles, one per grid z
+  int n_tt = 1, tt = 16;               // default token tiles (each plan may choose its own)
   token_tiles(n_mma, &n_tt, &tt);
-  const int T_tile = std::min(T, tt);
   const int nq = Q + 2 * KV;
-  const GemmPlan p_qkv = plan_gemm(fp, nq, w, tt, T_tile, true, false, n_tt);
-  const GemmPlan p_o = plan_gemm(fp, w, Q, tt, T_tile, true, false, n_tt);
-  const GemmPlan p_gu = plan_gemm(fp, 2 * F, w, tt, T_tile, false, fp->mlp_f8, n_tt);
-  const GemmPlan p_dn = plan_gemm(fp, w, F, tt, T_tile, true, fp->mlp_f8, n_tt);
+  const GemmPlan p_qkv = plan_suffix(fp, nq, w, n_mma, T, true, false);
+  const GemmPlan p_o = plan_suffix(fp, w, Q, n_mma, T, true, false);
+  const GemmPlan p_gu = plan_suffix(fp, 2 * F, w, n_mma, T, false, fp->mlp_f8);
+  const GemmPlan p_dn = plan_suffix(fp, w, F, n_mma, T, true, fp->mlp_f8);
   const int nk = P + S;
   const int nchunk = attn_chunks(fp, nk, k.n_q_heads * G);
   if (!(p_qkv.valid && p_o.valid && p_gu.valid && p_dn.valid) ||
@@ -2401,8 +2437,9 @@ rtv_status layers_impl(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     const GemmPlan* pls[4] = {&p_qkv, &p_o, &p_gu, &p_dn};
     const char* nm[4] = {"qkv", "o", "gu", "down"};
     for (int i = 0; i < 4; ++i)
-      fprintf(stderr, "[rtv] T=%d %s: tiles=%d cluster=%d kslice=%d stages=%d smem=%d\n", T, nm[i], pls[i]->n_tiles,
-              pls[i]->cs, pls[i]->kslice, pls[i]->stages, pls[i]->smem);
+      fprintf(stderr, "[rtv] T=%d %s: tiles=%d token_tiles=%d x %d cluster=%d kslice=%d stages=%d smem=%d\n", T,
+              nm[i], pls[i]->n_tiles, pls[i]->n_tt, pls[i]->tt, pls[i]->cs, pls[i]->kslice, pls[i]->stages,
+              pls[i]->smem);
     fprintf(stderr, "[rtv] gemm clusters that fit (size: two-per-SM budget / whole smem):");
     for (int cs = 1; cs <= 16; cs <<= 1) fprintf(stderr, " %d: %d/%d", cs, fp->gemm_fit_small[cs], fp->gemm_fit_large[cs]);
     fprintf(stderr, "\n");
@@ -2488,10 +2525,10 @@ rtv_status layers_impl(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
   const bool tracing = fp->trace_armed && fp->trace != nullptr;
   fp->trace_armed = false;
   if (tracing) {
-    fp->trace_ctas[0] = std::min(512, p_qkv.n_tiles * p_qkv.cs * n_tt);
-    fp->trace_ctas[1] = std::min(512, p_o.n_tiles * p_o.cs * n_tt);
-    fp->trace_ctas[2] = std::min(512, p_gu.n_tiles * p_gu.cs * n_tt);
-    fp->trace_ctas[3] = std::min(512, p_dn.n_tiles * p_dn.cs * n_tt);
+    fp->trace_ctas[0] = std::min(512, p_qkv.n_tiles * p_qkv.cs * p_qkv.n_tt);
+    fp->trace_ctas[1] = std::min(512, p_o.n_tiles * p_o.cs * p_o.n_tt);
+    fp->trace_ctas[2] = std::min(512, p_gu.n_tiles * p_gu.cs * p_gu.n_tt);
+    fp->trace_ctas[3] = std::min(512, p_dn.n_tiles * p_dn.cs * p_dn.n_tt);
     fp->trace_ctas[4] = std::min(512, tc_att ? (ntp + 1) * (k.n_q_heads / 2) * G : nchunk * k.n_q_heads * G);
   }
   auto tr = [&](int l, int i) -> unsigned long long* {
