@@ -114,6 +114,18 @@ def test_pi0_bf16_batch_two_matches_oracle(cuda_ok):
     assert bf16_tolerance_ok(got, ref)
 
 
+@pytest.mark.parametrize("batch", [3, 4, 5])
+def test_pi0_bf16_small_batches_token_tiling(cuda_ok, batch):
+    """153, 204 and 255 token rows: each projection picks its own token tiling
+    (1-4 tiles, the last one ragged) with its split; over the 816-token prefix
+    the attention grid (14 key tiles x 4 head pairs x batch) exceeds the SM
+    count, so it takes the compact two-CTAs-per-SM layout."""
+    cfg = get_config("pi0-bf16", n_layers=2)
+    got, ref, path = run_denoise(cfg, batch=batch, n_steps=2)
+    assert path == "tcgen05"
+    assert bf16_tolerance_ok(got, ref), (rel_l2(got, ref), np.max(np.abs(got - ref)))
+
+
 def test_pi0_bf16_batch_sixteen_token_tiles(cuda_ok):
     """16 chunks = 816 token rows: four token tiles of the projections (the
     MMA N is at most 256), sixteen suffix groups in the attention."""
