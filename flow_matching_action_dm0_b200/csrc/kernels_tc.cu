@@ -120,6 +120,12 @@ struct GemmArgs {
   int seq;                    // QKV: tokens of one sequence -- RoPE position and ks/vs row are t % seq, the
                               // sequence t / seq (= S for suffixes; the prefix length for a prefix)
   int kv_prefix;              // QKV with qt set: keys and values still go to ks / vs rows, not to kts / vts
+  // QKV writing keys and values as rows of a cached prefix (ks / vs): when
+  // set, also its tensor-core tiles, keys [seq][Hkv][ntile_max][64][D] and
+  // values transposed [seq][Hkv][ntile_max][D][64] (the layout the attention reads)
+  __nv_bfloat16* pkt;
+  __nv_bfloat16* pvt;
+  int ntile_max;
   // Per-layer time modulator (each suffix group g = t / S reads its own row):
   int g_stride;               // O, DOWN: the next norm's gain is g_next + g * g_stride (0: one gain for all)
   const float* sb;            // QKV, GU: added after the 1/rms factor, sb[g * sb_stride + natural row]
@@ -640,6 +646,23 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_tc_kernel(const GemmArgs
             else dst = a.vs + (((size_t)sq * a.Hkv + (hh - a.Hq - a.Hkv)) * a.kv_rows + sp) * a.D;
             *reinterpret_cast<uint32_t*>(dst + d1) = ptx::pack_bf16x2(y1.x, y1.y);
             *reinterpret_cast<uint32_t*>(dst + d2) = ptx::pack_bf16x2(y2.x, y2.y);
+            if (a.pkt && hh >= a.Hq) {   // the same key or value in the prefix's tiles
+              const bool is_k = hh < a.Hq + a.Hkv;
+              const int kh = is_k ? hh - a.Hq : hh - a.Hq - a.Hkv;
+              const size_t tile = ((size_t)sq * a.Hkv + kh) * a.ntile_max + (sp >> 6);
+              const int key = sp & 63;
+              if (is_k) {
+                __nv_bfloat16* kt = a.pkt + tile * 64 * a.D;
+                *reinterpret_cast<uint32_t*>(kt + ts_offset(key, d1, 64)) = ptx::pack_bf16x2(y1.x, y1.y);
+                *reinterpret_cast<uint32_t*>(kt + ts_offset(key, d2, 64)) = ptx::pack_bf16x2(y2.x, y2.y);
+              } else {
+                __nv_bfloat16* vt = a.pvt + tile * 64 * a.D;
+                vt[ts_offset(d1, key, a.D)] = __float2bfloat16_rn(y1.x);
+                vt[ts_offset(d1 + 1, key, a.D)] = __float2bfloat16_rn(y1.y);
+                vt[ts_offset(d2, key, a.D)] = __float2bfloat16_rn(y2.x);
+                vt[ts_offset(d2 + 1, key, a.D)] = __float2bfloat16_rn(y2.y);
+              }
+            }
           }
         }
       }
@@ -982,6 +1005,10 @@ struct AttnTcArgs {
   unsigned long long* trace;  // optional phase stamps [cta][kTraceRow], or nullptr
   long long timeout_ns;
   int S, P, Hq, Hkv, pbs, mask_mode, ntile_max, n_mma;
+  // 1: the prefix tiles are written by the kernel just before this one (the
+  // draft model's visual keys and values), so they are requested only after
+  // the dependency wait; 0: they were written before it and are requested first
+  int prefix_after_wait;
   float scale_log2;
 };
 
@@ -1062,12 +1089,14 @@ __global__ void __launch_bounds__(256, 2) attn_tc_kernel(const AttnTcArgs a) {
   const size_t kv_tile = suffix_tile ? (size_t)g * a.Hkv + kvh
                                      : ((size_t)(g * a.pbs) * a.Hkv + kvh) * a.ntile_max + rank;
   const __nv_bfloat16* vsrc = (suffix_tile ? a.vts : a.pvt) + kv_tile * 64 * D;
-  if (tid == 0 && !suffix_tile) {
+  auto load_prefix_tile = [&]() {
     ptx::mbar_expect_tx(&bars[0], (uint32_t)(COMPACT ? KB : KB + VB));
     ptx::bulk_load(Ks, a.pkt + kv_tile * 64 * D, (uint32_t)KB, &bars[0]);
     if (!COMPACT) ptx::bulk_load(Vs, vsrc, (uint32_t)VB, &bars[0]);
-  }
+  };
+  if (tid == 0 && !suffix_tile && !a.prefix_after_wait) load_prefix_tile();
   ptx::pdl_wait();
+  if (tid == 0 && !suffix_tile && a.prefix_after_wait) load_prefix_tile();
   if (trace && tid == 0) trace[1] = ptx::globaltimer();
   bool ok = true;
   if (tid == 0) {
@@ -2219,12 +2248,20 @@ rtv_status fast_block_prefix(rtv_ctx* ctx, const __nv_bfloat16* vis, int n_vis, 
   a.w_tile0 = 0;
   a.nt_base = ctx->Q / 128;
   a.eps = k.rms_eps;
+  // the tensor-core attention's tiles of the visual keys and values straight
+  // from the epilogue (no separate tiling pass over the cache)
+  const bool tiles = fp->tc_attn && (n_vis + 63) / 64 <= fp->ntile_max;
+  if (tiles) {
+    a.pkt = fp->pkt;
+    a.pvt = fp->pvt;
+    a.ntile_max = fp->ntile_max;
+  }
   if (e == cudaSuccess) e = launch_gemm<GM_QKV>(a, p, st);
   if (e != cudaSuccess) {
     ctx->last_error = std::string("visual-token projection launch: ") + cudaGetErrorString(e);
     return RTV_ERR_CUDA;
   }
-  return fast_prefix_update(ctx, batch, n_vis, st);
+  return tiles ? RTV_OK : fast_prefix_update(ctx, batch, n_vis, st);
 }
 
 rtv_status fast_block_embed(rtv_ctx* ctx, const float* rows, int n_src_rows, int G, cudaStream_t st) {
@@ -2519,6 +2556,9 @@ rtv_status layers_impl(rtv_ctx* ctx, int G, int P, int prefix_batch_stride, cons
     atc.ntile_max = fp->ntile_max;
     atc.n_mma = n_mma;
     atc.scale_log2 = at.scale_log2;
+    // a bare block's cached prefix (the draft's visual keys and values) is
+    // written by the kernel just before the layers
+    atc.prefix_after_wait = ctx->block_only ? 1 : 0;
   }
   const size_t ptile_layer = (size_t)k.max_batch * k.n_kv_heads * fp->ntile_max * 64 * D;
 
