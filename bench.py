@@ -98,8 +98,8 @@ def algorithmic_bytes_per_step(cfg, batch=1):
 # launches of a chunk with the L2 carried between kernels (profiles/dram_traffic_pi0-bf16_full_depth.md).  The
 # figure holds for the kernel sources it was taken on, identified by their SHA-256; after any change to them the
 # bench reports null until the capture is taken again.
-TRAFFIC_PI0_BF16 = {"bytes_per_chunk": 6445402624,
-                    "kernel_sources_sha256": "40bed238e85f5651098f690b4a1e9ba5db03b27a1b685b6b38713eba2ee4320b"}
+TRAFFIC_PI0_BF16 = {"bytes_per_chunk": 6436925184,
+                    "kernel_sources_sha256": "c2d3101a5c66b9f059bae20464169b3afb1e7a8780188a8b1b2f640ec3843f1e"}
 
 
 def kernel_sources_sha256():
